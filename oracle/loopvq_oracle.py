@@ -304,12 +304,12 @@ def decode_attn_ref(q: np.ndarray, win_K: np.ndarray, win_V: np.ndarray,
 # Written from the layout text of include/loopvq.h, independently of the
 # library's own code. The pool is
 #     [n_layers][n_kv_heads][n_loop_groups][n_pages][2 (K, V)][plane]
-# with a plane of page_tokens * J bytes. Inside a plane, tokens come in
-# blocks of 32. Inside a block, bytes are grouped in granules of GR bytes
-# (GR = 16 if J % 16 == 0, else 8 if J % 8 == 0, else 4) laid out
-#     [J / GR granules][32 tokens][GR bytes],
-# and the J index bytes of token slot i are rotated: group j sits at byte
-# position (j - (i mod 32)) mod J of that token's row.
+# with a plane of page_tokens * J bytes. Inside a plane, token slots come in
+# blocks of LB = floor(32/J)*J. Inside a block, bytes are grouped in granules
+# of GR bytes (GR = 16 if J % 16 == 0, else 8 if J % 8 == 0, else 4) laid out
+#     [J / GR granules][LB slots][GR bytes],
+# and the J index bytes of slot i are rotated: group j sits at byte position
+# (j - (i mod LB)) mod J of that slot's row.
 
 def pool_granule(J: int) -> int:
     if J % 16 == 0:
@@ -321,13 +321,21 @@ def pool_granule(J: int) -> int:
     raise ValueError("J = head_dim / c must be a multiple of 4")
 
 
+def rotation_block(J: int) -> int:
+    """LB: slots per rotation block, the largest multiple of J not above 32."""
+    if J > 32:
+        raise ValueError("J above 32 is not part of the format")
+    return (32 // J) * J
+
+
 def plane_offset(slot: int, j: int, J: int) -> int:
     """Byte offset of group ``j`` of token slot ``slot`` inside a plane."""
     gr = pool_granule(J)
-    blk, lane = divmod(slot, 32)
-    pos = (j - lane) % J
+    lb = rotation_block(J)
+    blk, rot = divmod(slot, lb)
+    pos = (j - rot) % J
     gran, byte = divmod(pos, gr)
-    return blk * 32 * J + gran * 32 * gr + lane * gr + byte
+    return blk * lb * J + gran * lb * gr + rot * gr + byte
 
 
 def pack_pages(idx_K: np.ndarray, idx_V: np.ndarray, pages: list[int],
@@ -346,6 +354,39 @@ def pack_pages(idx_K: np.ndarray, idx_V: np.ndarray, pages: list[int],
             out[pg, 0, off] = idx_K[v, j]
             out[pg, 1, off] = idx_V[v, j]
     return out
+
+
+def plane_offsets(slots: np.ndarray, J: int) -> np.ndarray:
+    """Array form of ``plane_offset``: ``[n]`` slots -> ``[n][J]`` offsets."""
+    gr = pool_granule(J)
+    lb = rotation_block(J)
+    slots = np.asarray(slots, dtype=np.int64)[:, None]
+    j = np.arange(J, dtype=np.int64)[None, :]
+    blk, rot = slots // lb, slots % lb
+    pos = (j - rot) % J
+    return blk * lb * J + (pos // gr) * lb * gr + rot * gr + pos % gr
+
+
+def pack_sequence(pool: np.ndarray, idx: np.ndarray, block_row: np.ndarray,
+                  page_tokens: int, kv: int) -> None:
+    """Write one sequence's indices ``idx [n][J]`` of one (layer, head, loop
+    group) into ``pool [n_pages][2][page_tokens*J]`` (in place) for K
+    (``kv = 0``) or V (``kv = 1``), following ``block_row`` (its page table
+    row)."""
+    n, J = idx.shape
+    v = np.arange(n, dtype=np.int64)
+    phys = np.asarray(block_row, dtype=np.int64)[v // page_tokens]
+    off = plane_offsets(v % page_tokens, J)
+    pool[phys[:, None], kv, off] = idx
+
+
+def unpack_sequence(pool: np.ndarray, n: int, J: int, block_row: np.ndarray,
+                    page_tokens: int, kv: int) -> np.ndarray:
+    """Inverse of ``pack_sequence``."""
+    v = np.arange(n, dtype=np.int64)
+    phys = np.asarray(block_row, dtype=np.int64)[v // page_tokens]
+    off = plane_offsets(v % page_tokens, J)
+    return pool[phys[:, None], kv, off]
 
 
 def unpack_pages(page_array: np.ndarray, pages: list[int], n: int,

@@ -303,13 +303,28 @@ def test_short_context_is_plain_attention():
 # states it): a hand-worked table of offsets plus a bijection check.
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("J", [12, 16, 24, 32, 8, 4])
+@pytest.mark.parametrize("J", [12, 16, 24, 32, 8, 4, 20, 28])
 def test_plane_offsets_form_a_bijection(J):
+    n = 3 * O.rotation_block(J)
     seen = set()
-    for slot in range(64):
+    for slot in range(n):
         for j in range(J):
             seen.add(O.plane_offset(slot, j, J))
-    assert seen == set(range(64 * J))
+    assert seen == set(range(n * J))
+
+
+@pytest.mark.parametrize("J", [12, 16, 24, 32, 8])
+def test_rotation_spreads_lanes_over_distinct_columns(J):
+    # at every step s, the slots of one block read distinct (replica, group)
+    # pairs, each group appearing floor(32/J) times: the property the format
+    # exists for.
+    lb = O.rotation_block(J)
+    for s in range(J):
+        cols = []
+        for rot in range(lb):
+            pos_of = {(j - rot) % J: j for j in range(J)}
+            cols.append((rot // J, pos_of[s]))
+        assert len(set(cols)) == lb
 
 
 def test_plane_offsets_hand_worked():
@@ -321,17 +336,18 @@ def test_plane_offsets_hand_worked():
     assert O.plane_offset(1, 0, 32) == 512 + 16 + 15
     # slot 33 is lane 1 of block 1 (1024 B in): group 1 -> 1024 + 16.
     assert O.plane_offset(33, 1, 32) == 1024 + 16
-    # J=12, granule 4. slot 2, group 0 -> pos 10 -> granule 2 (2*128), lane 2 (8), byte 2.
-    assert O.plane_offset(2, 0, 12) == 256 + 8 + 2
-    # J=12, slot 31 (lane 31), group 7 -> pos (7-31) mod 12 = 0 -> 31*4.
-    assert O.plane_offset(31, 7, 12) == 124
+    # J=12: LB=24, granule 4. slot 2, group 0 -> pos 10 -> granule 2
+    # (2*24*4 = 192), row 2 (8), byte 2.
+    assert O.plane_offset(2, 0, 12) == 192 + 8 + 2
+    # J=12, slot 31 is row 7 of block 1 (24*12 = 288 B in): group 7 -> pos 0.
+    assert O.plane_offset(31, 7, 12) == 288 + 28
     # J=24, granule 8. slot 5, group 6 -> pos 1 -> 5*8 + 1.
     assert O.plane_offset(5, 6, 24) == 41
 
 
 def test_pack_unpack_round_trip():
     r = _rng(19)
-    J, Pg, n = 12, 64, 150
+    J, Pg, n = 12, 96, 250
     iK = r.integers(0, 256, size=(n, J)).astype(np.uint8)
     iV = r.integers(0, 256, size=(n, J)).astype(np.uint8)
     pages = [4, 0, 2]
@@ -341,3 +357,22 @@ def test_pack_unpack_round_trip():
     np.testing.assert_array_equal(k2, iK)
     np.testing.assert_array_equal(v2, iV)
     assert not arr[1].any() and not arr[3].any()
+
+
+@pytest.mark.parametrize("J", [12, 16, 32, 24])
+def test_vector_packer_matches_scalar_packer(J):
+    r = _rng(20)
+    Pg = 2 * O.rotation_block(J) if O.rotation_block(J) != 32 else 64
+    n = 3 * Pg - 5
+    iK = r.integers(0, 256, size=(n, J)).astype(np.uint8)
+    iV = r.integers(0, 256, size=(n, J)).astype(np.uint8)
+    pages = [3, 1, 0]
+    ref = O.pack_pages(iK, iV, pages, 4, Pg)
+    pool = np.zeros((4, 2, Pg * J), dtype=np.uint8)
+    O.pack_sequence(pool, iK, np.array(pages), Pg, 0)
+    O.pack_sequence(pool, iV, np.array(pages), Pg, 1)
+    np.testing.assert_array_equal(pool, ref)
+    np.testing.assert_array_equal(O.unpack_sequence(pool, n, J, np.array(pages), Pg, 1), iV)
+    for s in range(0, Pg, 7):
+        np.testing.assert_array_equal(O.plane_offsets(np.array([s]), J)[0],
+                                      [O.plane_offset(s, j, J) for j in range(J)])
