@@ -1,0 +1,19 @@
+"""LoopVQ decode hot path for NVIDIA B200 (sm_100a).
+
+The work happens in ``libloopvq.so`` (hand-written CUDA); this package only
+loads it and marshals arguments. Importing it without the built library
+raises ``ImportError``: there is no CPU fallback.
+"""
+from .binding import (  # noqa: F401
+    LOOPVQ_DTYPE_BF16,
+    LOOPVQ_DTYPE_F32,
+    LoopVQConfig,
+    LoopVQError,
+    loopvq_bf16_decode_attn,
+    loopvq_bf16_decode_workspace_bytes,
+    loopvq_cache_layout,
+    loopvq_decode_attn,
+    loopvq_decode_workspace_bytes,
+    loopvq_encode,
+    loopvq_status_string,
+)

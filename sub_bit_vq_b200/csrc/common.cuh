@@ -1,0 +1,50 @@
+// Device helpers shared by the LoopVQ kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace loopvq {
+
+constexpr int kE = 256;           // centroids (8-bit index)
+constexpr int kRowStride = 32;    // floats per row of the [E][32] shared tables
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz.f32); relative error
+// about 2^-22, far inside the attention tolerances. Inputs here are <= 0 or
+// small positive, so no overflow.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
+  return __uint_as_float(bits16 << 16);
+}
+
+// Unpack a 32-bit word holding two bf16 values (low half first).
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Byte k (0..3) of a 32-bit word, as an integer.
+__device__ __forceinline__ uint32_t byte_of(uint32_t w, int k) {
+  return __byte_perm(w, 0u, 0x4440u | (uint32_t)k);
+}
+
+}  // namespace loopvq

@@ -1,0 +1,151 @@
+// Nearest-centroid encoder, direct form (sm_100a CUDA cores).
+//
+// One CTA = (tile of 128 tokens, channel group j, kv-head h). The CTA stages
+// the E x D codebook of (layer, h, gamma, K/V, j) in shared memory as
+// [E][D] (every thread then reads the same codeword: broadcast), and each
+// thread encodes one token's sub-vector
+//     s[tau*c + ch] = x[tau][n][h][j*c + ch],   tau < g, ch < c
+// by scanning all 256 codewords with the float32 weighted squared distance
+// sum_i w_i (s_i - C[e]_i)^2, keeping the first minimum (smallest index on
+// exact ties). The index byte goes to the rotated slot position of the pool.
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace loopvq {
+namespace {
+
+constexpr int kEncThreads = 128;
+
+struct EncodeParams {
+  const uint16_t* x;            // bf16 bits
+  int64_t x_loop_stride, x_token_stride;
+  const float* w;               // nullable
+  int64_t w_loop_stride, w_token_stride;
+  const float* cb;              // codebooks at (layer, head 0, gamma, kv, tau 0)
+  int64_t cb_stride_head, cb_stride_loop;
+  const int64_t* slot_mapping;
+  uint8_t* pool;                // pool at (layer, head 0, gamma)
+  int64_t pool_stride_head, page_bytes, plane_bytes;
+  int64_t n_slots;              // n_pages * Pg
+  int n_tokens, d, Pg, J, LB, GR, kv;
+};
+
+template <int C, int G>
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams p) {
+  constexpr int D = C * G;
+  __shared__ __align__(16) float cbs[kE * D];
+  const int j = blockIdx.y, h = blockIdx.z;
+  const float* cb = p.cb + h * p.cb_stride_head;
+  for (int i = threadIdx.x; i < kE * D; i += kEncThreads) {
+    const int e = i / D, k = i % D, tau = k / C, ch = k % C;
+    cbs[i] = cb[tau * p.cb_stride_loop + (static_cast<int64_t>(j) * kE + e) * C + ch];
+  }
+  __syncthreads();
+  const int n = blockIdx.x * kEncThreads + threadIdx.x;
+  if (n >= p.n_tokens) return;
+  const int64_t slot = p.slot_mapping[n];
+  if (slot < 0 || slot >= p.n_slots) return;
+
+  float s[D], w[D];
+#pragma unroll
+  for (int tau = 0; tau < G; ++tau) {
+    const uint16_t* xr = p.x + tau * p.x_loop_stride + n * p.x_token_stride +
+                         static_cast<int64_t>(h) * p.d + j * C;
+#pragma unroll
+    for (int ch = 0; ch < C; ++ch) s[tau * C + ch] = bf16_bits_to_float(xr[ch]);
+    if (p.w != nullptr) {
+      const float* wr = p.w + tau * p.w_loop_stride + n * p.w_token_stride +
+                        static_cast<int64_t>(h) * p.d + j * C;
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = wr[ch];
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = 1.f;
+    }
+  }
+
+  float best = INFINITY;
+  int best_e = 0;
+#pragma unroll 2
+  for (int e = 0; e < kE; ++e) {
+    const float4* c4 = reinterpret_cast<const float4*>(cbs + e * D);
+    float dist = 0.f;
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) {
+      const float4 cw = c4[k];
+      const float d0 = s[4 * k] - cw.x, d1 = s[4 * k + 1] - cw.y;
+      const float d2 = s[4 * k + 2] - cw.z, d3 = s[4 * k + 3] - cw.w;
+      dist = fmaf(w[4 * k] * d0, d0, dist);
+      dist = fmaf(w[4 * k + 1] * d1, d1, dist);
+      dist = fmaf(w[4 * k + 2] * d2, d2, dist);
+      dist = fmaf(w[4 * k + 3] * d3, d3, dist);
+    }
+    if (dist < best) {
+      best = dist;
+      best_e = e;
+    }
+  }
+
+  const int64_t page = slot / p.Pg;
+  const int sl = static_cast<int>(slot % p.Pg);
+  const int blk = sl / p.LB, rot = sl % p.LB;
+  int pos = j - rot % p.J;
+  if (pos < 0) pos += p.J;
+  const int64_t off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR +
+                      rot * p.GR + pos % p.GR;
+  p.pool[h * p.pool_stride_head + page * p.page_bytes + p.kv * p.plane_bytes + off] =
+      static_cast<uint8_t>(best_e);
+}
+
+template <int C, int G>
+loopvq_status launch_enc(const EncodeParams& p, int J, int H, cudaStream_t st) {
+  const dim3 grid((p.n_tokens + kEncThreads - 1) / kEncThreads, J, H);
+  encode_kernel<C, G><<<grid, kEncThreads, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+}
+
+}  // namespace
+
+loopvq_status launch_encode(const EncodeArgs& a) {
+  const Geometry& g = *a.geo;
+  EncodeParams p{};
+  p.x = static_cast<const uint16_t*>(a.x);
+  p.x_loop_stride = a.x_loop_stride;
+  p.x_token_stride = a.x_token_stride;
+  p.w = a.w;
+  p.w_loop_stride = a.w_loop_stride;
+  p.w_token_stride = a.w_token_stride;
+  p.cb = a.codebooks + a.layer * g.cb_stride_layer + a.gamma * g.cb_stride_group +
+         a.kv * g.cb_stride_kv;
+  p.cb_stride_head = g.cb_stride_head;
+  p.cb_stride_loop = g.cb_stride_loop;
+  p.slot_mapping = a.slot_mapping;
+  p.pool = a.pool + a.layer * g.pool_stride_layer + a.gamma * g.pool_stride_group;
+  p.pool_stride_head = g.pool_stride_head;
+  p.page_bytes = g.page_bytes;
+  p.plane_bytes = g.plane_bytes;
+  p.n_slots = static_cast<int64_t>(g.n_pages) * g.Pg;
+  p.n_tokens = a.n_tokens;
+  p.d = g.d;
+  p.Pg = g.Pg;
+  p.J = g.J;
+  p.LB = g.LB;
+  p.GR = g.GR;
+  p.kv = a.kv;
+  cudaStream_t st = static_cast<cudaStream_t>(a.stream);
+  switch (g.c * 100 + g.g) {
+    case 404: return launch_enc<4, 4>(p, g.J, g.Hkv, st);
+    case 804: return launch_enc<8, 4>(p, g.J, g.Hkv, st);
+    case 204: return launch_enc<2, 4>(p, g.J, g.Hkv, st);
+    case 402: return launch_enc<4, 2>(p, g.J, g.Hkv, st);
+    case 802: return launch_enc<8, 2>(p, g.J, g.Hkv, st);
+    case 208: return launch_enc<2, 8>(p, g.J, g.Hkv, st);
+    case 408: return launch_enc<4, 8>(p, g.J, g.Hkv, st);
+    case 401: return launch_enc<4, 1>(p, g.J, g.Hkv, st);
+    case 801: return launch_enc<8, 1>(p, g.J, g.Hkv, st);
+    default: return LOOPVQ_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace loopvq

@@ -1,0 +1,86 @@
+// Host-side declarations shared by the translation units of libloopvq.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "loopvq.h"
+
+namespace loopvq {
+
+// Everything derived from a validated loopvq_config.
+struct Geometry {
+  int L, Hkv, Hq, d, T, g, c, E, P, R, Pg, n_pages, max_batch, max_pages_per_seq;
+  int J, D, G, GR, LB, W;        // W = P + R window slots
+  int64_t plane_bytes, page_bytes;
+  int64_t pool_stride_group, pool_stride_head, pool_stride_layer;
+  int64_t cb_stride_loop, cb_stride_kv, cb_stride_group, cb_stride_head, cb_stride_layer;
+};
+
+// Validates `cfg` and fills `geo`. Pure host code.
+loopvq_status make_geometry(const loopvq_config* cfg, Geometry* geo);
+
+// Largest number of context splits the decode planner may use.
+int max_decode_splits(int pairs, int pages);
+
+// Number of multiprocessors of the current device (cached per device).
+// Returns 0 and sets *err when the runtime fails.
+int current_sm_count(loopvq_status* err);
+
+// Launchers (defined in the .cu files). All arguments are validated.
+struct DecodeArgs {
+  const Geometry* geo;
+  int layer, loop_step, batch, max_seq_len;
+  const void* q;
+  const uint8_t* pool;
+  const float* codebooks;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const void* win_k;
+  const void* win_v;
+  float sm_scale;
+  int out_dtype;
+  void* out;
+  float* lse;
+  void* workspace;
+  int splits;
+  void* stream;
+};
+loopvq_status launch_decode(const DecodeArgs& a);
+
+struct EncodeArgs {
+  const Geometry* geo;
+  int layer, gamma, kv, n_tokens;
+  const void* x;
+  int64_t x_loop_stride, x_token_stride;
+  const float* w;
+  int64_t w_loop_stride, w_token_stride;
+  const float* codebooks;
+  const int64_t* slot_mapping;
+  uint8_t* pool;
+  void* stream;
+};
+loopvq_status launch_encode(const EncodeArgs& a);
+
+struct Bf16DecodeArgs {
+  int batch, Hq, Hkv, d, max_seq_len;
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* seq_lens;
+  float sm_scale;
+  int out_dtype;
+  void* out;
+  float* lse;
+  void* workspace;
+  int splits;
+  void* stream;
+};
+loopvq_status launch_bf16_decode(const Bf16DecodeArgs& a);
+
+// Split-K merge of float32 partials [pairs][splits][d+2] (m in log2 units,
+// l, un-normalised o[d]) into out/lse.
+loopvq_status launch_merge(const float* partials, int pairs, int splits, int d, int out_dtype,
+                           void* out, float* lse, void* stream);
+
+}  // namespace loopvq
