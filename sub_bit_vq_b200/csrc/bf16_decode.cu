@@ -80,7 +80,10 @@ __global__ void __launch_bounds__(kBW * 32) bf16_decode_kernel(const Bf16Params 
   for (int i = 0; i < 8; ++i) o[i] = 0.f;
 
   constexpr int STEP = kBW * TPW;
-  for (int base = tok_lo + warp * TPW + tsub; base < tok_hi; base += STEP * kUnroll) {
+  // The loop bound is warp-uniform (base0 does not depend on the lane), so
+  // every lane runs the same trip count and reaches every full-mask shuffle.
+  for (int base0 = tok_lo + warp * TPW; base0 < tok_hi; base0 += STEP * kUnroll) {
+    const int base = base0 + tsub;
     uint4 kr[kUnroll], vr[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -106,20 +109,20 @@ __global__ void __launch_bounds__(kBW * 32) bf16_decode_kernel(const Bf16Params 
       }
 #pragma unroll
       for (int off = LPT / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      const float x = (t < tok_hi) ? dot : -INFINITY;
-      if (x == -INFINITY) continue;
-      const float mn = fmaxf(m, x);
-      const float sc = (m == mn) ? 1.f : fast_exp2(m - mn);
-      const float pr = fast_exp2(x - mn);
-      l = fmaf(l, sc, pr);
-      const uint32_t vw[4] = {vr[u].x, vr[u].y, vr[u].z, vr[u].w};
+      if (t < tok_hi) {                 // no shuffle inside this branch
+        const float mn = fmaxf(m, dot);
+        const float sc = (m == mn) ? 1.f : fast_exp2(m - mn);
+        const float pr = fast_exp2(dot - mn);
+        l = fmaf(l, sc, pr);
+        const uint32_t vw[4] = {vr[u].x, vr[u].y, vr[u].z, vr[u].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = bf16x2_to_float2(vw[i]);
-        o[2 * i] = fmaf(o[2 * i], sc, pr * f.x);
-        o[2 * i + 1] = fmaf(o[2 * i + 1], sc, pr * f.y);
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = bf16x2_to_float2(vw[i]);
+          o[2 * i] = fmaf(o[2 * i], sc, pr * f.x);
+          o[2 * i + 1] = fmaf(o[2 * i + 1], sc, pr * f.y);
+        }
+        m = mn;
       }
-      m = mn;
     }
   }
   // merge token groups of the warp

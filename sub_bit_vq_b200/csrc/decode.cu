@@ -167,14 +167,17 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
       uint32_t kw[NWORD], vw[NWORD];
       load_row<J, GR, LB>(kpl + blk * LB * J, lane, lane_live, kw);
       load_row<J, GR, LB>(vpl + blk * LB * J, lane, lane_live, vw);
-      float x = 0.f;
+      float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-      for (int s = 0; s < J; ++s) {
-        const uint32_t e = byte_of(kw[s >> 2], s & 3);
-        const int col = lane_live ? rbase + ((c0 + s) % J) : lane;
-        x += lut[e * kRowStride + col];
+      for (int s = 0; s < J; s += 2) {
+        const uint32_t e0 = byte_of(kw[s >> 2], s & 3);
+        const uint32_t e1 = byte_of(kw[(s + 1) >> 2], (s + 1) & 3);
+        const int col0 = lane_live ? rbase + ((c0 + s) % J) : lane;
+        const int col1 = lane_live ? rbase + ((c0 + s + 1) % J) : lane;
+        x0 += lut[e0 * kRowStride + col0];
+        x1 += lut[e1 * kRowStride + col1];
       }
-      x = valid ? x : -INFINITY;
+      const float x = valid ? x0 + x1 : -INFINITY;
       const float xm = warp_max(x);                  // finite: slot 0 of the block is valid
       if (xm > m_w + kRescaleSlack) {
         if (m_w != -INFINITY) {
@@ -193,12 +196,19 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
       }
       const float pr = valid ? fast_exp2(x - m_w) : 0.f;
       l_lane += pr;
+      // The J steps of one slot touch J distinct columns, hence J distinct
+      // words: issue every load before any store so the loads overlap.
+      int ha[J];
+      float hv[J];
 #pragma unroll
       for (int s = 0; s < J; ++s) {
         const uint32_t e = byte_of(vw[s >> 2], s & 3);
         const int col = lane_live ? rbase + ((c0 + s) % J) : lane;
-        my_hist[e * kRowStride + col] += pr;
+        ha[s] = e * kRowStride + col;
+        hv[s] = my_hist[ha[s]];
       }
+#pragma unroll
+      for (int s = 0; s < J; ++s) my_hist[ha[s]] = hv[s] + pr;
       __syncwarp();
     }
   }
