@@ -304,12 +304,14 @@ def decode_attn_ref(q: np.ndarray, win_K: np.ndarray, win_V: np.ndarray,
 # Written from the layout text of include/loopvq.h, independently of the
 # library's own code. The pool is
 #     [n_layers][n_kv_heads][n_loop_groups][n_pages][2 (K, V)][plane]
-# with a plane of page_tokens * J bytes. Inside a plane, token slots come in
-# blocks of LB = floor(32/J)*J. Inside a block, bytes are grouped in granules
-# of GR bytes (GR = 16 if J % 16 == 0, else 8 if J % 8 == 0, else 4) laid out
+# with a plane of page_tokens * J bytes.
+# K plane: token slots come in blocks of LB = floor(32/J)*J. Inside a block,
+# bytes are grouped in granules of GR bytes (GR = 16 if J % 16 == 0, else 8
+# if J % 8 == 0, else 4) laid out
 #     [J / GR granules][LB slots][GR bytes],
 # and the J index bytes of slot i are rotated: group j sits at byte position
 # (j - (i mod LB)) mod J of that slot's row.
+# V plane: group-major, (slot i, group j) at byte j * page_tokens + i.
 
 def pool_granule(J: int) -> int:
     if J % 16 == 0:
@@ -328,8 +330,11 @@ def rotation_block(J: int) -> int:
     return (32 // J) * J
 
 
-def plane_offset(slot: int, j: int, J: int) -> int:
-    """Byte offset of group ``j`` of token slot ``slot`` inside a plane."""
+def plane_offset(slot: int, j: int, J: int, kv: int = 0, page_tokens: int = 0) -> int:
+    """Byte offset of group ``j`` of token slot ``slot`` inside the K plane
+    (``kv = 0``) or the V plane (``kv = 1``, needs ``page_tokens``)."""
+    if kv == 1:
+        return j * page_tokens + slot
     gr = pool_granule(J)
     lb = rotation_block(J)
     blk, rot = divmod(slot, lb)
@@ -350,18 +355,19 @@ def pack_pages(idx_K: np.ndarray, idx_V: np.ndarray, pages: list[int],
         pg = pages[v // page_tokens]
         slot = v % page_tokens
         for j in range(J):
-            off = plane_offset(slot, j, J)
-            out[pg, 0, off] = idx_K[v, j]
-            out[pg, 1, off] = idx_V[v, j]
+            out[pg, 0, plane_offset(slot, j, J, 0)] = idx_K[v, j]
+            out[pg, 1, plane_offset(slot, j, J, 1, page_tokens)] = idx_V[v, j]
     return out
 
 
-def plane_offsets(slots: np.ndarray, J: int) -> np.ndarray:
+def plane_offsets(slots: np.ndarray, J: int, kv: int = 0, page_tokens: int = 0) -> np.ndarray:
     """Array form of ``plane_offset``: ``[n]`` slots -> ``[n][J]`` offsets."""
-    gr = pool_granule(J)
-    lb = rotation_block(J)
     slots = np.asarray(slots, dtype=np.int64)[:, None]
     j = np.arange(J, dtype=np.int64)[None, :]
+    if kv == 1:
+        return j * page_tokens + slots
+    gr = pool_granule(J)
+    lb = rotation_block(J)
     blk, rot = slots // lb, slots % lb
     pos = (j - rot) % J
     return blk * lb * J + (pos // gr) * lb * gr + rot * gr + pos % gr
@@ -376,7 +382,7 @@ def pack_sequence(pool: np.ndarray, idx: np.ndarray, block_row: np.ndarray,
     n, J = idx.shape
     v = np.arange(n, dtype=np.int64)
     phys = np.asarray(block_row, dtype=np.int64)[v // page_tokens]
-    off = plane_offsets(v % page_tokens, J)
+    off = plane_offsets(v % page_tokens, J, kv, page_tokens)
     pool[phys[:, None], kv, off] = idx
 
 
@@ -385,7 +391,7 @@ def unpack_sequence(pool: np.ndarray, n: int, J: int, block_row: np.ndarray,
     """Inverse of ``pack_sequence``."""
     v = np.arange(n, dtype=np.int64)
     phys = np.asarray(block_row, dtype=np.int64)[v // page_tokens]
-    off = plane_offsets(v % page_tokens, J)
+    off = plane_offsets(v % page_tokens, J, kv, page_tokens)
     return pool[phys[:, None], kv, off]
 
 
@@ -398,7 +404,6 @@ def unpack_pages(page_array: np.ndarray, pages: list[int], n: int,
         pg = pages[v // page_tokens]
         slot = v % page_tokens
         for j in range(J):
-            off = plane_offset(slot, j, J)
-            idx_K[v, j] = page_array[pg, 0, off]
-            idx_V[v, j] = page_array[pg, 1, off]
+            idx_K[v, j] = page_array[pg, 0, plane_offset(slot, j, J, 0)]
+            idx_V[v, j] = page_array[pg, 1, plane_offset(slot, j, J, 1, page_tokens)]
     return idx_K, idx_V

@@ -304,12 +304,13 @@ def test_short_context_is_plain_attention():
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("J", [12, 16, 24, 32, 8, 4, 20, 28])
-def test_plane_offsets_form_a_bijection(J):
+@pytest.mark.parametrize("kv", [0, 1])
+def test_plane_offsets_form_a_bijection(J, kv):
     n = 3 * O.rotation_block(J)
     seen = set()
     for slot in range(n):
         for j in range(J):
-            seen.add(O.plane_offset(slot, j, J))
+            seen.add(O.plane_offset(slot, j, J, kv, n))
     assert seen == set(range(n * J))
 
 
@@ -343,6 +344,9 @@ def test_plane_offsets_hand_worked():
     assert O.plane_offset(31, 7, 12) == 288 + 28
     # J=24, granule 8. slot 5, group 6 -> pos 1 -> 5*8 + 1.
     assert O.plane_offset(5, 6, 24) == 41
+    # V plane is group-major: slot 5, group 3 with 64-slot pages -> 3*64 + 5.
+    assert O.plane_offset(5, 3, 32, 1, 64) == 197
+    assert O.plane_offset(95, 11, 12, 1, 96) == 11 * 96 + 95
 
 
 def test_pack_unpack_round_trip():
@@ -374,5 +378,6 @@ def test_vector_packer_matches_scalar_packer(J):
     np.testing.assert_array_equal(pool, ref)
     np.testing.assert_array_equal(O.unpack_sequence(pool, n, J, np.array(pages), Pg, 1), iV)
     for s in range(0, Pg, 7):
-        np.testing.assert_array_equal(O.plane_offsets(np.array([s]), J)[0],
-                                      [O.plane_offset(s, j, J) for j in range(J)])
+        for kv in (0, 1):
+            np.testing.assert_array_equal(O.plane_offsets(np.array([s]), J, kv, Pg)[0],
+                                          [O.plane_offset(s, j, J, kv, Pg) for j in range(J)])
