@@ -57,7 +57,7 @@ enum { LOOPVQ_DTYPE_BF16 = 0, LOOPVQ_DTYPE_F32 = 1 };
  * head_dim <= 256; chan_group in {1,2,4,8,16} dividing head_dim; J = d/c a
  * multiple of 4 and at most 32; n_loops % loop_group == 0; D = c*g <= 32;
  * n_centroids == 256; page_tokens a multiple of the rotation block
- * LB = floor(32/J)*J and at most 256; n_q_heads % n_kv_heads == 0.
+ * LB = floor(32/J)*J and of 16, at most 256; n_q_heads % n_kv_heads == 0.
  */
 typedef struct {
   uint32_t struct_size;      /* sizeof(loopvq_config) */
@@ -83,18 +83,23 @@ typedef struct {
  * Index pool (uint8), row-major
  *     [L][Hkv][G][n_pages][2 (K, V)][plane]
  * with one plane = Pg*J bytes holding the K (or V) indices of Pg token
- * slots. Inside a plane, slots come in blocks of LB = floor(32/J)*J. Inside
- * a block the bytes are stored in granules of GR bytes (GR = 16 if
- * J % 16 == 0, else 8 if J % 8 == 0, else 4) as
+ * slots.
+ *
+ * K plane: slots come in blocks of LB = floor(32/J)*J. Inside a block the
+ * bytes are stored in granules of GR bytes (GR = 16 if J % 16 == 0, else 8
+ * if J % 8 == 0, else 4) as
  *     [J/GR granules][LB slots][GR bytes],
  * and the J index bytes of slot i are rotated: the index of channel group
  * j sits at byte position (j - (i mod LB)) mod J of that slot's row. So
- * the byte offset of (slot i, group j) inside a plane is
+ * the byte offset of (slot i, group j) inside the K plane is
  *     (i/LB)*LB*J + (pos/GR)*LB*GR + (i%LB)*GR + pos%GR,
  *     pos = (j - i%LB) mod J.
  * The rotation lets one warp lane per slot read its own row while the
  * lanes of a warp touch distinct columns of a [E][32] table, which keeps
  * shared memory free of bank conflicts.
+ *
+ * V plane: group-major, the byte of (slot i, group j) is at j*Pg + i. One
+ * lane per channel group then owns one column of the value histogram.
  *
  * Quantised token v of a sequence (v = position - P, for positions
  * P .. N-R-1) lives in page block_table[b][v / Pg], slot v % Pg.

@@ -70,7 +70,7 @@ loopvq_status make_geometry(const loopvq_config* cfg, Geometry* geo) {
   if (g.W > 256) return LOOPVQ_ERR_UNSUPPORTED;
   g.GR = (g.J % 16 == 0) ? 16 : (g.J % 8 == 0) ? 8 : 4;
   g.LB = (32 / g.J) * g.J;
-  if (g.Pg % g.LB != 0 || g.Pg > 256) return LOOPVQ_ERR_UNSUPPORTED;
+  if (g.Pg % g.LB != 0 || g.Pg % 16 != 0 || g.Pg > 256) return LOOPVQ_ERR_UNSUPPORTED;
   g.plane_bytes = static_cast<int64_t>(g.Pg) * g.J;
   g.page_bytes = 2 * g.plane_bytes;
   if (!mul_ok(g.page_bytes, g.n_pages, &g.pool_stride_group)) return LOOPVQ_ERR_INVALID_ARG;

@@ -1,19 +1,22 @@
 // Fused LoopVQ decode attention over the packed index cache (sm_100a).
 //
-// One CTA = one (sequence b, query head hq, context split). Per CTA:
-//   1. q (bf16) -> shared, pre-scaled by sm_scale*log2(e) so scores live in
-//      log2 units and every exponential is a single ex2.
-//   2. Key lookup table LUT[e][col] = q_j . C_K[j][e][tau][:] for the
-//      loop-tau codebook slice ([E][32] float, column = replica*J + j).
-//   3. Each warp streams whole index pages. One lane owns one token slot:
-//      it loads its token's rotated row of J key bytes and J value bytes
-//      (16-, 8- or 4-byte granules), sums J LUT entries to get the score,
-//      and adds p = 2^(x - m) into its warp's private value histogram
-//      W[e][col]. Because rows are rotated by the slot's lane, the 32 lanes
-//      of a warp touch 32 distinct columns at every step: no bank conflicts
-//      and no two lanes on one histogram word.
-//   4. The window tokens (bf16 prefix + recent) are scored densely by
-//      split 0.
+// One CTA = one (sequence b, query head hq, context split), 6 warps. Per CTA:
+//   1. q (bf16) is pre-scaled by sm_scale*log2(e): scores live in log2
+//      units and every exponential is one ex2.
+//   2. Key lookup table LUT[e][col] = q_j . C_K[j][e][tau][:] from the
+//      loop-tau codebook slice ([E][32] float; column = replica*J + j).
+//   3. The bf16 window tokens (prefix + recent) are scored densely
+//      (split 0 only) and kept as a (m, l, o) partial.
+//   4. Each warp streams blocks of LB token slots. Key pass: lane = slot;
+//      the slot's rotated row of J key bytes gives J LUT reads that hit J
+//      distinct columns across the warp (no bank conflicts); the score is a
+//      per-lane sum. Value pass: lane = (replica, channel group) and owns
+//      one column of its warp's private histogram W[e][col]; it adds
+//      p = 2^(x - m) of its J slots at the rows given by the group-major
+//      value bytes, two slots per step with an equality check so that two
+//      updates of one word in a step merge. No lane ever writes another
+//      lane's column, so no atomics and no warp-level ordering are needed.
+//      Index bytes are prefetched 4 blocks ahead into registers.
 //   5. Warps are merged, the histogram is contracted with the loop-tau value
 //      codebook slice (o[j*c+ch] = sum_e W[e][j] C_V[j][e][tau][ch]) and the
 //      split writes (m, l, o[d]) to the workspace.
@@ -29,8 +32,9 @@
 namespace loopvq {
 namespace {
 
-constexpr int kNW = 4;                  // warps per CTA, each with its own histogram
+constexpr int kNW = 6;                  // warps per CTA, one value histogram each
 constexpr int kThreads = kNW * 32;
+constexpr int kDepth = 4;               // blocks in flight per warp
 constexpr float kRescaleSlack = 8.0f;   // log2 units a new maximum may exceed m before rescaling
 
 struct DecodeParams {
@@ -51,51 +55,76 @@ struct DecodeParams {
   float scale_log2;
 };
 
-// Loads the rotated row (J bytes) of `row` (this lane's slot) from a block
-// of LB slots stored as [J/GR][LB][GR] bytes. `words[k]` = row bytes 4k..4k+3.
-template <int J, int GR, int LB>
-__device__ __forceinline__ void load_row(const uint8_t* block, int row, bool live,
-                                         uint32_t (&words)[J / 4]) {
-  constexpr int NG = J / GR;
-  if (!live) {
+template <int J>
+struct Traits {
+  static constexpr int R = 32 / J;      // replicas of each column per table row
+  static constexpr int LB = R * J;      // slots per block
+  static constexpr int GR = (J % 16 == 0) ? 16 : (J % 8 == 0) ? 8 : 4;   // granule
+  static constexpr int NWORD = J / 4;   // words per lane per plane and block
+};
+
+template <int J>
+struct BlockRegs {
+  uint32_t k[J / 4];   // this lane's rotated key row (lane = slot)
+  uint32_t v[J / 4];   // this lane's value bytes: group j, J consecutive slots
+  bool ok;             // page present (same value in every lane)
+};
+
+template <int GR>
+__device__ __forceinline__ void load_words(const uint8_t* src, uint32_t* w, int nwords) {
+  // nwords is a compile-time multiple of GR/4 at every call site
 #pragma unroll
-    for (int k = 0; k < J / 4; ++k) words[k] = 0u;
-    return;
-  }
-#pragma unroll
-  for (int gi = 0; gi < NG; ++gi) {
-    const uint8_t* src = block + gi * LB * GR + row * GR;
+  for (int i = 0; i < nwords; i += GR / 4) {
     if constexpr (GR == 16) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src));
-      words[gi * 4 + 0] = v.x;
-      words[gi * 4 + 1] = v.y;
-      words[gi * 4 + 2] = v.z;
-      words[gi * 4 + 3] = v.w;
+      const uint4 t = __ldcs(reinterpret_cast<const uint4*>(src + 4 * i));
+      w[i] = t.x; w[i + 1] = t.y; w[i + 2] = t.z; w[i + 3] = t.w;
     } else if constexpr (GR == 8) {
-      const uint2 v = __ldcs(reinterpret_cast<const uint2*>(src));
-      words[gi * 2 + 0] = v.x;
-      words[gi * 2 + 1] = v.y;
+      const uint2 t = __ldcs(reinterpret_cast<const uint2*>(src + 4 * i));
+      w[i] = t.x; w[i + 1] = t.y;
     } else {
-      words[gi] = __ldcs(reinterpret_cast<const unsigned int*>(src));
+      w[i] = __ldcs(reinterpret_cast<const unsigned int*>(src + 4 * i));
+    }
+  }
+}
+
+// Loads block `blk` of the page at `kpl` (K plane; the V plane follows).
+template <int J>
+__device__ __forceinline__ void load_block(const uint8_t* kpl, int64_t plane_bytes, int Pg, int blk,
+                                           int lane, BlockRegs<J>& r) {
+  using T = Traits<J>;
+  if (lane < T::LB) {
+    // K: rotated rows, [J/GR][LB][GR] per block
+#pragma unroll
+    for (int gi = 0; gi < J / T::GR; ++gi)
+      load_words<T::GR>(kpl + blk * T::LB * J + gi * T::LB * T::GR + lane * T::GR,
+                        r.k + gi * (T::GR / 4), T::GR / 4);
+    // V: group-major; lane = (replica rr, group j) reads J slots of group j
+    const int rr = lane / J, j = lane % J;
+    load_words<T::GR>(kpl + plane_bytes + static_cast<int64_t>(j) * Pg + blk * T::LB + rr * J, r.v,
+                      T::NWORD);
+  } else {
+#pragma unroll
+    for (int i = 0; i < T::NWORD; ++i) {
+      r.k[i] = 0u;
+      r.v[i] = 0u;
     }
   }
 }
 
 template <int J, int C>
 __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodeParams p) {
+  using T = Traits<J>;
   constexpr int d = J * C;
-  constexpr int R = 32 / J;                  // replicas of each column per row
-  constexpr int LB = R * J;                  // slots per rotation block
-  constexpr int GR = (J % 16 == 0) ? 16 : (J % 8 == 0) ? 8 : 4;
-  constexpr int NWORD = J / 4;
+  constexpr int R = T::R, LB = T::LB;
+  constexpr int OPT = (d + kThreads - 1) / kThreads;   // output channels per thread
 
   extern __shared__ __align__(16) float smem[];
   float* lut = smem;                                   // [E][32]
   float* hist = lut + kE * kRowStride;                 // [kNW][E][32]
-  float* qs = hist + kNW * kE * kRowStride;            // [256]
-  float* xwin = qs + 256;                              // [256]
-  float* owin = xwin + 256;                            // [256]
-  float* wstat = owin + 256;                           // [2*kNW]
+  float* pbuf = hist + kNW * kE * kRowStride;          // [kNW][32]
+  float* wstat = pbuf + kNW * 32;                      // [2*kNW]
+  float* qs = hist;                                    // scratch before the histograms are zeroed
+  float* xwin = hist + 256;
 
   const int split = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -114,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   const float* cbk = p.cb_k + hkv * p.cb_stride_head;
   const float* cbv = p.cb_v + hkv * p.cb_stride_head;
 
-  // ---- key lookup table and histogram reset ----------------------------
+  // ---- key lookup table; window scores -----------------------------------
   {
     const int j = lane % J;
     const bool live = lane < LB;
@@ -122,8 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
 #pragma unroll
     for (int ch = 0; ch < C; ++ch) qj[ch] = qs[j * C + ch];
     const float* src = cbk + static_cast<size_t>(j) * kE * C;
-    constexpr int EPW = kE / kNW;
-    for (int e = warp * EPW; e < (warp + 1) * EPW; ++e) {
+    for (int e = warp; e < kE; e += kNW) {
       float v = 0.f;
       if constexpr (C % 4 == 0) {
 #pragma unroll
@@ -140,76 +168,156 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
       }
       lut[e * kRowStride + lane] = live ? v : 0.f;
     }
+  }
+  if (n_win > 0) {
+    const uint16_t* wk =
+        p.win_k + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
+    for (int t = warp; t < n_win; t += kNW) {
+      float acc = 0.f;
+      for (int ch = lane; ch < d; ch += 32)
+        acc = fmaf(qs[ch], bf16_bits_to_float(wk[t * d + ch]), acc);
+      acc = warp_sum(acc);
+      if (lane == 0) xwin[t] = acc;
+    }
+  }
+  __syncthreads();
+  float m_win = -INFINITY, l_win = 0.f;
+  float owin[OPT];
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) owin[k] = 0.f;
+  if (n_win > 0) {
+    for (int t = 0; t < n_win; ++t) m_win = fmaxf(m_win, xwin[t]);
+    for (int t = 0; t < n_win; ++t) l_win += fast_exp2(xwin[t] - m_win);
+    const uint16_t* wv =
+        p.win_v + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+      const int ch = tid + k * kThreads;
+      if (ch < d) {
+        float o = 0.f;
+        for (int t = 0; t < n_win; ++t)
+          o = fmaf(fast_exp2(xwin[t] - m_win), bf16_bits_to_float(wv[t * d + ch]), o);
+        owin[k] = o;
+      }
+    }
+  }
+  __syncthreads();                                      // scratch (qs, xwin) no longer read
+  {
     float4* h4 = reinterpret_cast<float4*>(hist + warp * kE * kRowStride);
     for (int i = lane; i < kE * kRowStride / 4; i += 32) h4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __syncthreads();
+  __syncwarp();
 
-  // ---- stream index pages -----------------------------------------------
-  const bool lane_live = lane < LB;
+  // ---- stream index blocks ------------------------------------------------
   const int c0 = lane % J;
   const int rbase = lane - c0;
+  const bool lane_live = lane < LB;
   float* my_hist = hist + warp * kE * kRowStride;
+  float* my_p = pbuf + warp * 32;
   float m_w = -INFINITY;
   float l_lane = 0.f;
   const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
   const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages_per_seq;
 
-  for (int pg = pg_lo + warp; pg < pg_hi; pg += kNW) {
-    const int phys = bt[pg];
-    if (phys < 0 || phys >= p.n_pages) continue;     // absent page: warp-uniform skip
-    const uint8_t* kpl = pool_h + static_cast<int64_t>(phys) * p.page_bytes;
-    const uint8_t* vpl = kpl + p.plane_bytes;
+  const int my_first = pg_lo + warp;
+  const int n_my_pages = (pg_hi > my_first) ? (pg_hi - my_first + kNW - 1) / kNW : 0;
+  const int bpp = p.Pg / LB;                            // blocks per page
+  const int n_blocks = n_my_pages * bpp;
+
+  // page table window: lane l holds the physical page of this warp's page
+  // index i0 + l (cur) and i0 + 32 + l (nxt)
+  int i0 = 0;
+  auto bt_entry = [&](int i) -> int {
+    return (i < n_my_pages) ? bt[my_first + i * kNW] : -1;
+  };
+  int bt_cur = bt_entry(lane);
+  int bt_nxt = bt_entry(32 + lane);
+
+  BlockRegs<J> ring[kDepth];
+  // Issues the loads of block k (page index k / bpp of this warp).
+  auto issue = [&](int k, BlockRegs<J>& r) {
+    const int pi = k / bpp;
+    if (pi >= i0 + 32) {                                // warp-uniform
+      bt_cur = bt_nxt;
+      i0 += 32;
+      bt_nxt = bt_entry(i0 + 32 + lane);
+    }
+    const int phys = __shfl_sync(0xffffffffu, bt_cur, pi - i0);
+    r.ok = phys >= 0 && phys < p.n_pages;
+    if (!r.ok) {                                        // absent page: read nothing
+#pragma unroll
+      for (int i = 0; i < T::NWORD; ++i) {
+        r.k[i] = 0u;
+        r.v[i] = 0u;
+      }
+      return;
+    }
+    load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, p.Pg, k % bpp,
+                  lane, r);
+  };
+
+  auto process = [&](int k, const BlockRegs<J>& r) {
+    const int pi = k / bpp, blk = k % bpp;
+    const int pg = my_first + pi * kNW;
     const int valid_in_page = min(p.Pg, n_vq - pg * p.Pg);
-    const int nblk = (valid_in_page + LB - 1) / LB;
-    for (int blk = 0; blk < nblk; ++blk) {
-      const bool valid = lane_live && (blk * LB + lane) < valid_in_page;
-      uint32_t kw[NWORD], vw[NWORD];
-      load_row<J, GR, LB>(kpl + blk * LB * J, lane, lane_live, kw);
-      load_row<J, GR, LB>(vpl + blk * LB * J, lane, lane_live, vw);
-      float x0 = 0.f, x1 = 0.f;
+    const int base = blk * LB;
+    if (base >= valid_in_page || !r.ok) return;         // warp-uniform
+    // key pass: lane = slot
+    float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-      for (int s = 0; s < J; s += 2) {
-        const uint32_t e0 = byte_of(kw[s >> 2], s & 3);
-        const uint32_t e1 = byte_of(kw[(s + 1) >> 2], (s + 1) & 3);
-        const int col0 = lane_live ? rbase + ((c0 + s) % J) : lane;
-        const int col1 = lane_live ? rbase + ((c0 + s + 1) % J) : lane;
-        x0 += lut[e0 * kRowStride + col0];
-        x1 += lut[e1 * kRowStride + col1];
+    for (int s = 0; s < J; s += 2) {
+      const uint32_t e0 = byte_of(r.k[s >> 2], s & 3);
+      const uint32_t e1 = byte_of(r.k[(s + 1) >> 2], (s + 1) & 3);
+      const int col0 = lane_live ? rbase + ((c0 + s) % J) : lane;
+      const int col1 = lane_live ? rbase + ((c0 + s + 1) % J) : lane;
+      x0 += lut[e0 * kRowStride + col0];
+      x1 += lut[e1 * kRowStride + col1];
+    }
+    const bool valid = lane_live && (base + lane) < valid_in_page;
+    const float x = valid ? x0 + x1 : -INFINITY;
+    const float xm = warp_max(x);                       // finite: slot 0 of the block is valid
+    if (xm > m_w + kRescaleSlack) {                     // warp-uniform
+      if (m_w != -INFINITY) {
+        const float f = fast_exp2(m_w - xm);
+        for (int e = 0; e < kE; ++e) my_hist[e * kRowStride + lane] *= f;   // own column
+        l_lane *= f;
       }
-      const float x = valid ? x0 + x1 : -INFINITY;
-      const float xm = warp_max(x);                  // finite: slot 0 of the block is valid
-      if (xm > m_w + kRescaleSlack) {
-        if (m_w != -INFINITY) {
-          const float f = fast_exp2(m_w - xm);
-          __syncwarp();
-          float4* h4 = reinterpret_cast<float4*>(my_hist);
-          for (int i = lane; i < kE * kRowStride / 4; i += 32) {
-            float4 t = h4[i];
-            t.x *= f; t.y *= f; t.z *= f; t.w *= f;
-            h4[i] = t;
-          }
-          __syncwarp();
-          l_lane *= f;
-        }
-        m_w = xm;
-      }
-      const float pr = valid ? fast_exp2(x - m_w) : 0.f;
-      l_lane += pr;
-      // The J steps of one slot touch J distinct columns, hence J distinct
-      // words: issue every load before any store so the loads overlap.
-      int ha[J];
-      float hv[J];
+      m_w = xm;
+    }
+    const float pr = valid ? fast_exp2(x - m_w) : 0.f;
+    l_lane += pr;
+    my_p[lane] = pr;
+    __syncwarp();
+    // value pass: lane = (replica, group) owns column `lane`; slots rr*J + i
+    if (lane_live) {
+      const float* pp = my_p + (lane / J) * J;
 #pragma unroll
-      for (int s = 0; s < J; ++s) {
-        const uint32_t e = byte_of(vw[s >> 2], s & 3);
-        const int col = lane_live ? rbase + ((c0 + s) % J) : lane;
-        ha[s] = e * kRowStride + col;
-        hv[s] = my_hist[ha[s]];
+      for (int i = 0; i < J; i += 2) {
+        const uint32_t ea = byte_of(r.v[i >> 2], i & 3);
+        const uint32_t eb = byte_of(r.v[(i + 1) >> 2], (i + 1) & 3);
+        const float2 pab = *reinterpret_cast<const float2*>(pp + i);
+        float* wa = my_hist + ea * kRowStride + lane;
+        float* wb = my_hist + eb * kRowStride + lane;
+        const float va = *wa, vb = *wb;
+        const bool same = (ea == eb);
+        const float na = va + (same ? pab.x + pab.y : pab.x);
+        const float nb = same ? na : vb + pab.y;
+        *wa = na;
+        *wb = nb;
       }
+    }
+    __syncwarp();                                       // my_p is rewritten by the next block
+  };
+
 #pragma unroll
-      for (int s = 0; s < J; ++s) my_hist[ha[s]] = hv[s] + pr;
-      __syncwarp();
+  for (int u = 0; u < kDepth - 1; ++u)
+    if (u < n_blocks) issue(u, ring[u]);
+  for (int k0 = 0; k0 < n_blocks; k0 += kDepth) {
+#pragma unroll
+    for (int u = 0; u < kDepth; ++u) {
+      const int k = k0 + u;
+      if (k + kDepth - 1 < n_blocks) issue(k + kDepth - 1, ring[(u + kDepth - 1) % kDepth]);
+      if (k < n_blocks) process(k, ring[u]);
     }
   }
   const float l_w = warp_sum(l_lane);
@@ -217,40 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
     wstat[warp] = m_w;
     wstat[kNW + warp] = l_w;
   }
-
-  // ---- bf16 window tokens (split 0) -----------------------------------
-  if (n_win > 0) {
-    const uint16_t* wk =
-        p.win_k + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
-    for (int t = warp; t < n_win; t += kNW) {
-      float acc = 0.f;
-      for (int ch = lane; ch < d; ch += 32) acc = fmaf(qs[ch], bf16_bits_to_float(wk[t * d + ch]), acc);
-      acc = warp_sum(acc);
-      if (lane == 0) xwin[t] = acc;
-    }
-  }
   __syncthreads();
-  float m_win = -INFINITY;
-  float l_win = 0.f;
-  if (n_win > 0) {
-    for (int t = 0; t < n_win; ++t) m_win = fmaxf(m_win, xwin[t]);
-    for (int t = 0; t < n_win; ++t) l_win += fast_exp2(xwin[t] - m_win);
-    const uint16_t* wv =
-        p.win_v + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
-    for (int ch = tid; ch < d; ch += kThreads) {
-      float o = 0.f;
-      for (int t = 0; t < n_win; ++t)
-        o = fmaf(fast_exp2(xwin[t] - m_win), bf16_bits_to_float(wv[t * d + ch]), o);
-      owin[ch] = o;
-    }
-  }
 
   // ---- merge warps, contract the histogram -----------------------------
   float M = m_win;
 #pragma unroll
   for (int w = 0; w < kNW; ++w) M = fmaxf(M, wstat[w]);
   float* part = p.partials + (static_cast<size_t>(b * p.Hq + hq) * p.S + split) * (d + 2);
-  if (M == -INFINITY) {                               // no token in this split
+  if (M == -INFINITY) {                                 // no token in this split
     for (int i = tid; i < d + 2; i += kThreads) part[i] = (i == 0) ? -INFINITY : 0.f;
     return;
   }
@@ -279,18 +361,22 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
     }
   }
   __syncthreads();
-  for (int o = tid; o < d; o += kThreads) {
-    const int j = o / C, ch = o % C;
-    const float* src = cbv + static_cast<size_t>(j) * kE * C + ch;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int e = 0; e < kE; ++e) {
-      float wsum = 0.f;
 #pragma unroll
-      for (int r = 0; r < R; ++r) wsum += hist[e * kRowStride + r * J + j];
-      acc = fmaf(wsum, __ldg(src + e * C), acc);
+  for (int k = 0; k < OPT; ++k) {
+    const int o = tid + k * kThreads;
+    if (o < d) {
+      const int j = o / C, ch = o % C;
+      const float* src = cbv + static_cast<size_t>(j) * kE * C + ch;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < kE; ++e) {
+        float wsum = 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) wsum += hist[e * kRowStride + r * J + j];
+        acc = fmaf(wsum, __ldg(src + e * C), acc);
+      }
+      part[2 + o] = acc + f_win * owin[k];
     }
-    part[2 + o] = acc + ((n_win > 0) ? f_win * owin[o] : 0.f);
   }
   if (tid == 0) {
     part[0] = M;
@@ -339,8 +425,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ pa
 }
 
 constexpr size_t decode_smem_bytes() {
-  return (static_cast<size_t>(kE) * kRowStride * (1 + kNW) + 256 * 3 + 2 * kNW) * sizeof(float);
+  return (static_cast<size_t>(kE) * kRowStride * (1 + kNW) + kNW * 32 + 2 * kNW) * sizeof(float);
 }
+static_assert(decode_smem_bytes() <= 227 * 1024, "decode kernel shared memory above 227 KB");
 
 template <int J, int C>
 loopvq_status launch_vq(const DecodeParams& p, dim3 grid, cudaStream_t st) {

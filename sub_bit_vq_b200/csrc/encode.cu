@@ -89,11 +89,16 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
 
   const int64_t page = slot / p.Pg;
   const int sl = static_cast<int>(slot % p.Pg);
-  const int blk = sl / p.LB, rot = sl % p.LB;
-  int pos = j - rot % p.J;
-  if (pos < 0) pos += p.J;
-  const int64_t off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR +
-                      rot * p.GR + pos % p.GR;
+  int64_t off;
+  if (p.kv == 0) {                          // K plane: rotated slot rows
+    const int blk = sl / p.LB, rot = sl % p.LB;
+    int pos = j - rot % p.J;
+    if (pos < 0) pos += p.J;
+    off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR + rot * p.GR +
+          pos % p.GR;
+  } else {                                  // V plane: group-major
+    off = static_cast<int64_t>(j) * p.Pg + sl;
+  }
   p.pool[h * p.pool_stride_head + page * p.page_bytes + p.kv * p.plane_bytes + off] =
       static_cast<uint8_t>(best_e);
 }

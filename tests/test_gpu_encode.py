@@ -46,7 +46,7 @@ def _gpu_indices(pool, s, layer, gamma, kv, slots):
         if sl < 0:
             continue
         page, slot = divmod(int(sl), s.page_tokens)
-        off = O.plane_offsets(np.array([slot]), s.J)[0]
+        off = O.plane_offsets(np.array([slot]), s.J, kv, s.page_tokens)[0]
         for h in range(s.n_kv_heads):
             out[n, h] = pool[layer, h, gamma, page, kv, off]
     return out
@@ -98,7 +98,7 @@ def test_weighted_encode_with_skips_and_paging(per_token):
     written = set()
     for sl in slots[keep]:
         page, slot = divmod(int(sl), s.page_tokens)
-        for o in O.plane_offsets(np.array([slot]), s.J)[0]:
+        for o in O.plane_offsets(np.array([slot]), s.J, kv, s.page_tokens)[0]:
             written.add((page, int(o)))
     mask = np.zeros((n_pages, s.page_tokens * s.J), dtype=bool)
     for page, o in written:
