@@ -47,4 +47,16 @@ __device__ __forceinline__ uint32_t byte_of(uint32_t w, int k) {
   return __byte_perm(w, 0u, 0x4440u | (uint32_t)k);
 }
 
+// 16-byte asynchronous global -> shared copy (cp.async, L2 only). Both
+// addresses must be 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
+
+// Waits until every cp.async this thread issued has landed in shared memory.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
 }  // namespace loopvq

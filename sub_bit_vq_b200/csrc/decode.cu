@@ -1,12 +1,15 @@
 // Fused LoopVQ decode attention over the packed index cache (sm_100a).
 //
-// One CTA = one (sequence b, query head hq, context split), 6 warps. Per CTA:
-//   1. q (bf16) is pre-scaled by sm_scale*log2(e): scores live in log2
-//      units and every exponential is one ex2.
-//   2. Key lookup table LUT[e][col] = q_j . C_K[j][e][tau][:] from the
-//      loop-tau codebook slice ([E][32] float; column = replica*J + j).
-//   3. The bf16 window tokens (prefix + recent) are scored densely
-//      (split 0 only) and kept as a (m, l, o) partial.
+// One CTA = one (sequence b, query head hq, context split), 6 warps, one CTA
+// per SM (the per-warp value histograms fill shared memory). Per CTA:
+//   1. The first index blocks of every warp are requested (register ring),
+//      then the loop-tau key codebook slice is staged into shared memory
+//      with cp.async while q is pre-scaled by sm_scale*log2(e) (scores live
+//      in log2 units: every exponential is one ex2).
+//   2. Key lookup table LUT[e][col] = q_j . C_K[j][e][tau][:] ([E][32]
+//      float, column = replica*J + j), built from shared memory.
+//   3. Split 0 scores the bf16 window tokens (prefix + recent) densely and
+//      keeps them as a (m, l, o) partial.
 //   4. Each warp streams blocks of LB token slots. Key pass: lane = slot;
 //      the slot's rotated row of J key bytes gives J LUT reads that hit J
 //      distinct columns across the warp (no bank conflicts); the score is a
@@ -14,13 +17,13 @@
 //      one column of its warp's private histogram W[e][col]; it adds
 //      p = 2^(x - m) of its J slots at the rows given by the group-major
 //      value bytes, two slots per step with an equality check so that two
-//      updates of one word in a step merge. No lane ever writes another
-//      lane's column, so no atomics and no warp-level ordering are needed.
-//      Index bytes are prefetched 4 blocks ahead into registers.
-//   5. Warps are merged, the histogram is contracted with the loop-tau value
-//      codebook slice (o[j*c+ch] = sum_e W[e][j] C_V[j][e][tau][ch]) and the
-//      split writes (m, l, o[d]) to the workspace.
-// A second kernel merges the splits (log-sum-exp merge) into out and lse.
+//      updates of one word in a step merge. No lane writes another lane's
+//      column, so no atomics and no warp-level ordering are needed. Index
+//      bytes are prefetched kDepth blocks ahead into registers.
+//   5. Warps are merged, the loop-tau value codebook slice is staged into
+//      the freed histogram space and contracted with the histogram
+//      (o[j*c+ch] = sum_e W[e][j] C_V[j][e][tau][ch]); the split writes
+//      (m, l, o[d]) to the workspace. merge.cu combines the splits.
 
 #include <math.h>
 
@@ -35,6 +38,9 @@ namespace {
 constexpr int kNW = 6;                  // warps per CTA, one value histogram each
 constexpr int kThreads = kNW * 32;
 constexpr int kDepth = 4;               // blocks in flight per warp
+constexpr int kRegion = kE * kRowStride;  // floats in one [E][32] table (32 KB)
+constexpr int kStageRegions = 4;        // histogram regions 1..4 double as codebook staging
+constexpr int kWinChunk = 12;           // window tokens per warp per round of loads
 constexpr float kRescaleSlack = 8.0f;   // log2 units a new maximum may exceed m before rescaling
 
 struct DecodeParams {
@@ -72,7 +78,6 @@ struct BlockRegs {
 
 template <int GR>
 __device__ __forceinline__ void load_words(const uint8_t* src, uint32_t* w, int nwords) {
-  // nwords is a compile-time multiple of GR/4 at every call site
 #pragma unroll
   for (int i = 0; i < nwords; i += GR / 4) {
     if constexpr (GR == 16) {
@@ -93,12 +98,10 @@ __device__ __forceinline__ void load_block(const uint8_t* kpl, int64_t plane_byt
                                            int lane, BlockRegs<J>& r) {
   using T = Traits<J>;
   if (lane < T::LB) {
-    // K: rotated rows, [J/GR][LB][GR] per block
 #pragma unroll
     for (int gi = 0; gi < J / T::GR; ++gi)
       load_words<T::GR>(kpl + blk * T::LB * J + gi * T::LB * T::GR + lane * T::GR,
                         r.k + gi * (T::GR / 4), T::GR / 4);
-    // V: group-major; lane = (replica rr, group j) reads J slots of group j
     const int rr = lane / J, j = lane % J;
     load_words<T::GR>(kpl + plane_bytes + static_cast<int64_t>(j) * Pg + blk * T::LB + rr * J, r.v,
                       T::NWORD);
@@ -111,20 +114,54 @@ __device__ __forceinline__ void load_block(const uint8_t* kpl, int64_t plane_byt
   }
 }
 
+// Copies `nfloats` (multiple of 4) from global to shared with cp.async.
+__device__ __forceinline__ void stage_async(float* dst, const float* src, int nfloats, int tid) {
+  for (int i = tid * 4; i < nfloats; i += kThreads * 4) cp_async16(dst + i, src + i);
+}
+
+// sum_ch a[ch] * b[ch] for C channels held contiguously (16-byte aligned
+// when C % 4 == 0).
+template <int C>
+__device__ __forceinline__ float dot_c(const float* a, const float* b) {
+  float v = 0.f;
+  if constexpr (C % 4 == 0) {
+#pragma unroll
+    for (int ch = 0; ch < C; ch += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(a + ch);
+      const float4 y = *reinterpret_cast<const float4*>(b + ch);
+      v = fmaf(x.x, y.x, v);
+      v = fmaf(x.y, y.y, v);
+      v = fmaf(x.z, y.z, v);
+      v = fmaf(x.w, y.w, v);
+    }
+  } else {
+#pragma unroll
+    for (int ch = 0; ch < C; ++ch) v = fmaf(a[ch], b[ch], v);
+  }
+  return v;
+}
+
 template <int J, int C>
 __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodeParams p) {
   using T = Traits<J>;
   constexpr int d = J * C;
   constexpr int R = T::R, LB = T::LB;
   constexpr int OPT = (d + kThreads - 1) / kThreads;   // output channels per thread
+  constexpr int NPL = (d / 2 + 31) / 32;               // bf16 channel pairs per lane (window)
+  // channel groups per staging chunk: a [JC][E][C] slice fits regions 1..4
+  constexpr int JC = (J * kE * C <= kStageRegions * kRegion) ? J : (kStageRegions * kRegion) / (kE * C);
+  static_assert(J % JC == 0, "staging chunks must tile the channel groups");
 
   extern __shared__ __align__(16) float smem[];
   float* lut = smem;                                   // [E][32]
-  float* hist = lut + kE * kRowStride;                 // [kNW][E][32]
-  float* pbuf = hist + kNW * kE * kRowStride;          // [kNW][32]
+  float* hist = lut + kRegion;                         // [kNW][E][32]
+  float* pbuf = hist + kNW * kRegion;                  // [kNW][32]
   float* wstat = pbuf + kNW * 32;                      // [2*kNW]
-  float* qs = hist;                                    // scratch before the histograms are zeroed
-  float* xwin = hist + 256;
+  float* stage = hist + kRegion;                       // regions 1..4
+  // scratch inside region 0 until the histograms are zeroed
+  float* qs = hist;                                    // [256]
+  float* xwin = hist + 256;                            // [256]
+  float* opart = hist + 512;                           // [kNW][256]
 
   const int split = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -135,106 +172,26 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   const int pg_lo = split * p.pps;
   const int pg_hi = min(n_pg, pg_lo + p.pps);
   const int n_win = (split == 0) ? min(N, p.W) : 0;
-
-  const uint16_t* qp = p.q + (static_cast<size_t>(b) * p.Hq + hq) * d;
-  for (int i = tid; i < d; i += kThreads) qs[i] = bf16_bits_to_float(qp[i]) * p.scale_log2;
-  __syncthreads();
-
   const float* cbk = p.cb_k + hkv * p.cb_stride_head;
   const float* cbv = p.cb_v + hkv * p.cb_stride_head;
 
-  // ---- key lookup table; window scores -----------------------------------
-  {
-    const int j = lane % J;
-    const bool live = lane < LB;
-    float qj[C];
-#pragma unroll
-    for (int ch = 0; ch < C; ++ch) qj[ch] = qs[j * C + ch];
-    const float* src = cbk + static_cast<size_t>(j) * kE * C;
-    for (int e = warp; e < kE; e += kNW) {
-      float v = 0.f;
-      if constexpr (C % 4 == 0) {
-#pragma unroll
-        for (int ch = 0; ch < C; ch += 4) {
-          const float4 cw = __ldg(reinterpret_cast<const float4*>(src + e * C + ch));
-          v = fmaf(qj[ch], cw.x, v);
-          v = fmaf(qj[ch + 1], cw.y, v);
-          v = fmaf(qj[ch + 2], cw.z, v);
-          v = fmaf(qj[ch + 3], cw.w, v);
-        }
-      } else {
-#pragma unroll
-        for (int ch = 0; ch < C; ++ch) v = fmaf(qj[ch], __ldg(src + e * C + ch), v);
-      }
-      lut[e * kRowStride + lane] = live ? v : 0.f;
-    }
-  }
-  if (n_win > 0) {
-    const uint16_t* wk =
-        p.win_k + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
-    for (int t = warp; t < n_win; t += kNW) {
-      float acc = 0.f;
-      for (int ch = lane; ch < d; ch += 32)
-        acc = fmaf(qs[ch], bf16_bits_to_float(wk[t * d + ch]), acc);
-      acc = warp_sum(acc);
-      if (lane == 0) xwin[t] = acc;
-    }
-  }
-  __syncthreads();
-  float m_win = -INFINITY, l_win = 0.f;
-  float owin[OPT];
-#pragma unroll
-  for (int k = 0; k < OPT; ++k) owin[k] = 0.f;
-  if (n_win > 0) {
-    for (int t = 0; t < n_win; ++t) m_win = fmaxf(m_win, xwin[t]);
-    for (int t = 0; t < n_win; ++t) l_win += fast_exp2(xwin[t] - m_win);
-    const uint16_t* wv =
-        p.win_v + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
-#pragma unroll
-    for (int k = 0; k < OPT; ++k) {
-      const int ch = tid + k * kThreads;
-      if (ch < d) {
-        float o = 0.f;
-        for (int t = 0; t < n_win; ++t)
-          o = fmaf(fast_exp2(xwin[t] - m_win), bf16_bits_to_float(wv[t * d + ch]), o);
-        owin[k] = o;
-      }
-    }
-  }
-  __syncthreads();                                      // scratch (qs, xwin) no longer read
-  {
-    float4* h4 = reinterpret_cast<float4*>(hist + warp * kE * kRowStride);
-    for (int i = lane; i < kE * kRowStride / 4; i += 32) h4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  __syncwarp();
-
-  // ---- stream index blocks ------------------------------------------------
+  // ---- 1. request the first index blocks of this warp ---------------------
   const int c0 = lane % J;
   const int rbase = lane - c0;
   const bool lane_live = lane < LB;
-  float* my_hist = hist + warp * kE * kRowStride;
-  float* my_p = pbuf + warp * 32;
-  float m_w = -INFINITY;
-  float l_lane = 0.f;
   const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
   const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages_per_seq;
-
   const int my_first = pg_lo + warp;
   const int n_my_pages = (pg_hi > my_first) ? (pg_hi - my_first + kNW - 1) / kNW : 0;
   const int bpp = p.Pg / LB;                            // blocks per page
   const int n_blocks = n_my_pages * bpp;
-
   // page table window: lane l holds the physical page of this warp's page
   // index i0 + l (cur) and i0 + 32 + l (nxt)
   int i0 = 0;
-  auto bt_entry = [&](int i) -> int {
-    return (i < n_my_pages) ? bt[my_first + i * kNW] : -1;
-  };
+  auto bt_entry = [&](int i) -> int { return (i < n_my_pages) ? bt[my_first + i * kNW] : -1; };
   int bt_cur = bt_entry(lane);
   int bt_nxt = bt_entry(32 + lane);
-
   BlockRegs<J> ring[kDepth];
-  // Issues the loads of block k (page index k / bpp of this warp).
   auto issue = [&](int k, BlockRegs<J>& r) {
     const int pi = k / bpp;
     if (pi >= i0 + 32) {                                // warp-uniform
@@ -255,6 +212,158 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
     load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, p.Pg, k % bpp,
                   lane, r);
   };
+#pragma unroll
+  for (int u = 0; u < kDepth - 1; ++u)
+    if (u < n_blocks) issue(u, ring[u]);
+
+  // ---- 2. key lookup table (codebook staged in regions 1..4) ---------------
+  stage_async(stage, cbk, JC * kE * C, tid);
+  const uint16_t* qp = p.q + (static_cast<size_t>(b) * p.Hq + hq) * d;
+  for (int i = tid; i < d; i += kThreads) qs[i] = bf16_bits_to_float(qp[i]) * p.scale_log2;
+
+  // ---- 3. window keys: one round of loads per kWinChunk tokens per warp ---
+  uint32_t wv_reg[kWinChunk][NPL];                      // first chunk of window values
+  const uint16_t* wkb = p.win_k + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
+  const uint16_t* wvb = p.win_v + (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * d;
+  if (n_win > 0) {
+#pragma unroll
+    for (int i = 0; i < kWinChunk; ++i) {
+      const int t = warp + i * kNW;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const int pc = lane + 32 * k;                   // channel pair index
+        wv_reg[i][k] = (t < n_win && pc < d / 2)
+                           ? __ldg(reinterpret_cast<const unsigned int*>(wvb + t * d) + pc) : 0u;
+      }
+    }
+  }
+  __syncthreads();                                      // qs visible
+  for (int t0 = warp; t0 < n_win; t0 += kNW * kWinChunk) {
+    uint32_t kr[kWinChunk][NPL];
+#pragma unroll
+    for (int i = 0; i < kWinChunk; ++i) {
+      const int t = t0 + i * kNW;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const int pc = lane + 32 * k;
+        kr[i][k] = (t < n_win && pc < d / 2)
+                       ? __ldg(reinterpret_cast<const unsigned int*>(wkb + t * d) + pc) : 0u;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kWinChunk; ++i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const int pc = lane + 32 * k;
+        if (pc < d / 2) {
+          const float2 kv = bf16x2_to_float2(kr[i][k]);
+          acc = fmaf(qs[2 * pc], kv.x, fmaf(qs[2 * pc + 1], kv.y, acc));
+        }
+      }
+      acc = warp_sum(acc);
+      const int t = t0 + i * kNW;
+      if (lane == 0 && t < n_win) xwin[t] = acc;
+    }
+  }
+
+  // ---- LUT from the staged key codebook ----------------------------------
+  for (int j0 = 0; j0 < J; j0 += JC) {
+    if (j0 > 0) {
+      __syncthreads();                                  // previous chunk consumed
+      stage_async(stage, cbk + static_cast<size_t>(j0) * kE * C, JC * kE * C, tid);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // item = (e-tile of 32, step s): lane -> e = tile*32 + lane, group
+    // j0 + (lane + s) % JC; rotating the group keeps the table writes on
+    // distinct banks.
+    for (int item = warp; item < (kE / 32) * JC; item += kNW) {
+      const int tile = item / JC, s = item % JC;
+      const int e = tile * 32 + lane;
+      const int jj = (lane + s) % JC;
+      const int j = j0 + jj;
+      const float v = dot_c<C>(qs + j * C, stage + (static_cast<size_t>(jj) * kE + e) * C);
+#pragma unroll
+      for (int r = 0; r < R; ++r) lut[e * kRowStride + r * J + j] = v;
+    }
+  }
+  if (LB < 32) {                                        // columns no slot reads: keep them 0
+    for (int i = tid; i < kE * (32 - LB); i += kThreads)
+      lut[(i / (32 - LB)) * kRowStride + LB + i % (32 - LB)] = 0.f;
+  }
+  __syncthreads();                                      // xwin complete, LUT complete
+
+  // ---- window partial -----------------------------------------------------
+  float m_win = -INFINITY, l_win = 0.f;
+  float owin[OPT];
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) owin[k] = 0.f;
+  if (n_win > 0) {
+    for (int t = 0; t < n_win; ++t) m_win = fmaxf(m_win, xwin[t]);
+    for (int t = 0; t < n_win; ++t) l_win += fast_exp2(xwin[t] - m_win);
+    float oacc[NPL][2];
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) oacc[k][0] = oacc[k][1] = 0.f;
+    for (int t0 = warp; t0 < n_win; t0 += kNW * kWinChunk) {
+      uint32_t vr[kWinChunk][NPL];
+#pragma unroll
+      for (int i = 0; i < kWinChunk; ++i) {
+        const int t = t0 + i * kNW;
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) {
+          const int pc = lane + 32 * k;
+          vr[i][k] = (t0 == warp) ? wv_reg[i][k]
+                     : ((t < n_win && pc < d / 2)
+                            ? __ldg(reinterpret_cast<const unsigned int*>(wvb + t * d) + pc) : 0u);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kWinChunk; ++i) {
+        const int t = t0 + i * kNW;
+        const float w = (t < n_win) ? fast_exp2(xwin[t] - m_win) : 0.f;
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) {
+          const float2 vv = bf16x2_to_float2(vr[i][k]);
+          oacc[k][0] = fmaf(w, vv.x, oacc[k][0]);
+          oacc[k][1] = fmaf(w, vv.y, oacc[k][1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+      const int pc = lane + 32 * k;
+      if (pc < d / 2) {
+        opart[warp * 256 + 2 * pc] = oacc[k][0];
+        opart[warp * 256 + 2 * pc + 1] = oacc[k][1];
+      }
+    }
+  }
+  __syncthreads();
+  if (n_win > 0) {
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+      const int ch = tid + k * kThreads;
+      if (ch < d) {
+        float o = 0.f;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) o += opart[w * 256 + ch];
+        owin[k] = o;
+      }
+    }
+  }
+  __syncthreads();                                      // scratch in region 0 no longer read
+  {
+    float4* h4 = reinterpret_cast<float4*>(hist + warp * kRegion);
+    for (int i = lane; i < kRegion / 4; i += 32) h4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncwarp();
+
+  // ---- 4. stream index blocks --------------------------------------------
+  float* my_hist = hist + warp * kRegion;
+  float* my_p = pbuf + warp * 32;
+  float m_w = -INFINITY;
+  float l_lane = 0.f;
 
   auto process = [&](int k, const BlockRegs<J>& r) {
     const int pi = k / bpp, blk = k % bpp;
@@ -309,9 +418,6 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
     __syncwarp();                                       // my_p is rewritten by the next block
   };
 
-#pragma unroll
-  for (int u = 0; u < kDepth - 1; ++u)
-    if (u < n_blocks) issue(u, ring[u]);
   for (int k0 = 0; k0 < n_blocks; k0 += kDepth) {
 #pragma unroll
     for (int u = 0; u < kDepth; ++u) {
@@ -327,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   }
   __syncthreads();
 
-  // ---- merge warps, contract the histogram -----------------------------
+  // ---- 5. merge warps, contract the histogram -----------------------------
   float M = m_win;
 #pragma unroll
   for (int w = 0; w < kNW; ++w) M = fmaxf(M, wstat[w]);
@@ -347,11 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   L += f_win * l_win;
   {
     float4* h0 = reinterpret_cast<float4*>(hist);
-    for (int i = tid; i < kE * kRowStride / 4; i += kThreads) {
+    for (int i = tid; i < kRegion / 4; i += kThreads) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int w = 0; w < kNW; ++w) {
-        const float4 t = reinterpret_cast<const float4*>(hist + w * kE * kRowStride)[i];
+        const float4 t = reinterpret_cast<const float4*>(hist + w * kRegion)[i];
         acc.x = fmaf(f[w], t.x, acc.x);
         acc.y = fmaf(f[w], t.y, acc.y);
         acc.z = fmaf(f[w], t.z, acc.z);
@@ -360,23 +466,35 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
       h0[i] = acc;
     }
   }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < OPT; ++k) {
-    const int o = tid + k * kThreads;
-    if (o < d) {
-      const int j = o / C, ch = o % C;
-      const float* src = cbv + static_cast<size_t>(j) * kE * C + ch;
+  for (int j0 = 0; j0 < J; j0 += JC) {
+    __syncthreads();                                    // histogram merged / previous chunk used
+    stage_async(stage, cbv + static_cast<size_t>(j0) * kE * C, JC * kE * C, tid);
+    cp_async_wait_all();
+    __syncthreads();
+    // thread -> (group jj, channel ch); rows visited from e = jj so that the
+    // threads of a warp read different banks of the staged slice
+    for (int t = tid; t < JC * C; t += kThreads) {
+      const int jj = t / C, ch = t % C, j = j0 + jj;
+      const float* cv = stage + static_cast<size_t>(jj) * kE * C + ch;
       float acc = 0.f;
 #pragma unroll 8
-      for (int e = 0; e < kE; ++e) {
+      for (int i = 0; i < kE; ++i) {
+        const int e = (i + jj) & (kE - 1);
         float wsum = 0.f;
 #pragma unroll
         for (int r = 0; r < R; ++r) wsum += hist[e * kRowStride + r * J + j];
-        acc = fmaf(wsum, __ldg(src + e * C), acc);
+        acc = fmaf(wsum, cv[e * C], acc);
       }
-      part[2 + o] = acc + f_win * owin[k];
+      const int o = j * C + ch;
+      // the window part of channel o lives in thread o % kThreads, slot o / kThreads
+      part[2 + o] = acc;
     }
+  }
+  __syncthreads();                                      // every part[2 + o] written
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) {
+    const int o = tid + k * kThreads;
+    if (o < d && f_win != 0.f) part[2 + o] += f_win * owin[k];
   }
   if (tid == 0) {
     part[0] = M;
@@ -384,48 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   }
 }
 
-// (m, l, o) partials [pairs][S][d+2] -> out [pairs][d], lse [pairs].
-__global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ partials, int pairs,
-                                                    int S, int d, int out_dtype, void* out,
-                                                    float* lse) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x * 4 + warp;
-  if (pair >= pairs) return;
-  const int stride = d + 2;
-  const float* P = partials + static_cast<size_t>(pair) * S * stride;
-  float M = -INFINITY;
-  for (int s = lane; s < S; s += 32) M = fmaxf(M, P[s * stride]);
-  M = warp_max(M);
-  float L = 0.f;
-  if (M != -INFINITY) {
-    for (int s = lane; s < S; s += 32) {
-      const float m = P[s * stride];
-      if (m != -INFINITY) L += P[s * stride + 1] * fast_exp2(m - M);
-    }
-  }
-  L = warp_sum(L);
-  const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  for (int ch = lane; ch < d; ch += 32) {
-    float o = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const float m = P[s * stride];
-        if (m != -INFINITY) o = fmaf(P[s * stride + 2 + ch], fast_exp2(m - M), o);
-      }
-    }
-    o *= inv;
-    if (out_dtype == LOOPVQ_DTYPE_F32) {
-      static_cast<float*>(out)[static_cast<size_t>(pair) * d + ch] = o;
-    } else {
-      static_cast<__nv_bfloat16*>(out)[static_cast<size_t>(pair) * d + ch] = __float2bfloat16_rn(o);
-    }
-  }
-  if (lane == 0 && lse != nullptr)
-    lse[pair] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
-}
-
 constexpr size_t decode_smem_bytes() {
-  return (static_cast<size_t>(kE) * kRowStride * (1 + kNW) + kNW * 32 + 2 * kNW) * sizeof(float);
+  return (static_cast<size_t>(kRegion) * (1 + kNW) + kNW * 32 + 2 * kNW) * sizeof(float);
 }
 static_assert(decode_smem_bytes() <= 227 * 1024, "decode kernel shared memory above 227 KB");
 
@@ -448,14 +526,6 @@ loopvq_status launch_vq(const DecodeParams& p, dim3 grid, cudaStream_t st) {
 }
 
 }  // namespace
-
-loopvq_status launch_merge(const float* partials, int pairs, int splits, int d, int out_dtype,
-                           void* out, float* lse, void* stream) {
-  const dim3 grid((pairs + 3) / 4);
-  merge_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(partials, pairs, splits, d,
-                                                                     out_dtype, out, lse);
-  return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
-}
 
 loopvq_status launch_decode(const DecodeArgs& a) {
   const Geometry& g = *a.geo;
