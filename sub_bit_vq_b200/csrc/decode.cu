@@ -1,13 +1,14 @@
 // Fused LoopVQ decode attention over the packed index cache (sm_100a).
 //
-// One CTA = one (sequence b, query head hq, context split), 6 warps, one CTA
+// One CTA = one (sequence b, query head hq, context split), 5 warps, one CTA
 // per SM (the per-warp value histograms fill shared memory). Per CTA:
 //   1. The first index blocks of every warp are requested (register ring),
 //      then the loop-tau key codebook slice is staged into shared memory
 //      with cp.async while q is pre-scaled by sm_scale*log2(e) (scores live
 //      in log2 units: every exponential is one ex2).
-//   2. Key lookup table LUT[e][col] = q_j . C_K[j][e][tau][:] ([E][32]
-//      float, column = replica*J + j), built from shared memory.
+//   2. Key lookup table LUT[e][k] = q_j . C_K[j][e][tau][:] with j = k % J,
+//      [E][64] float (every group repeated along the row so that a lane's
+//      column lane + step never wraps), built from shared memory.
 //   3. Split 0 scores the bf16 window tokens (prefix + recent) densely and
 //      keeps them as a (m, l, o) partial.
 //   4. Each warp streams blocks of LB token slots. Key pass: lane = slot;
@@ -35,10 +36,12 @@
 namespace loopvq {
 namespace {
 
-constexpr int kNW = 6;                  // warps per CTA, one value histogram each
+constexpr int kNW = 5;                  // warps per CTA, one value histogram each
 constexpr int kThreads = kNW * 32;
 constexpr int kDepth = 4;               // blocks in flight per warp
 constexpr int kRegion = kE * kRowStride;  // floats in one [E][32] table (32 KB)
+constexpr int kLutRow = 64;             // LUT row: 64 columns, column k holds group k % J
+constexpr int kLutFloats = kE * kLutRow;  // 64 KB
 constexpr int kStageRegions = 4;        // histogram regions 1..4 double as codebook staging
 constexpr int kWinChunk = 12;           // window tokens per warp per round of loads
 constexpr float kRescaleSlack = 8.0f;   // log2 units a new maximum may exceed m before rescaling
@@ -153,8 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   static_assert(J % JC == 0, "staging chunks must tile the channel groups");
 
   extern __shared__ __align__(16) float smem[];
-  float* lut = smem;                                   // [E][32]
-  float* hist = lut + kRegion;                         // [kNW][E][32]
+  float* lut = smem;                                   // [E][64]
+  float* hist = lut + kLutFloats;                      // [kNW][E][32]
   float* pbuf = hist + kNW * kRegion;                  // [kNW][32]
   float* wstat = pbuf + kNW * 32;                      // [2*kNW]
   float* stage = hist + kRegion;                       // regions 1..4
@@ -176,8 +179,6 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   const float* cbv = p.cb_v + hkv * p.cb_stride_head;
 
   // ---- 1. request the first index blocks of this warp ---------------------
-  const int c0 = lane % J;
-  const int rbase = lane - c0;
   const bool lane_live = lane < LB;
   const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
   const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages_per_seq;
@@ -285,12 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
       const int j = j0 + jj;
       const float v = dot_c<C>(qs + j * C, stage + (static_cast<size_t>(jj) * kE + e) * C);
 #pragma unroll
-      for (int r = 0; r < R; ++r) lut[e * kRowStride + r * J + j] = v;
+      for (int k = j; k < kLutRow; k += J) lut[e * kLutRow + k] = v;
     }
-  }
-  if (LB < 32) {                                        // columns no slot reads: keep them 0
-    for (int i = tid; i < kE * (32 - LB); i += kThreads)
-      lut[(i / (32 - LB)) * kRowStride + LB + i % (32 - LB)] = 0.f;
   }
   __syncthreads();                                      // xwin complete, LUT complete
 
@@ -362,6 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   // ---- 4. stream index blocks --------------------------------------------
   float* my_hist = hist + warp * kRegion;
   float* my_p = pbuf + warp * 32;
+  const char* lut_bytes = reinterpret_cast<const char*>(lut);
+  char* hist_bytes = reinterpret_cast<char*>(my_hist);
+  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;   // fits one byte
+  const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;   // fits one byte
   float m_w = -INFINITY;
   float l_lane = 0.f;
 
@@ -371,23 +372,22 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
     const int valid_in_page = min(p.Pg, n_vq - pg * p.Pg);
     const int base = blk * LB;
     if (base >= valid_in_page || !r.ok) return;         // warp-uniform
-    // key pass: lane = slot
-    float x0 = 0.f, x1 = 0.f;
+    // key pass: lane = slot. Row byte s holds the index of group
+    // (lane + s) % J, which LUT column lane + s holds: one byte permute
+    // forms (e << 8) | lane*4 and the step goes into the load's offset.
+    float xa[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s = 0; s < J; s += 2) {
-      const uint32_t e0 = byte_of(r.k[s >> 2], s & 3);
-      const uint32_t e1 = byte_of(r.k[(s + 1) >> 2], (s + 1) & 3);
-      const int col0 = lane_live ? rbase + ((c0 + s) % J) : lane;
-      const int col1 = lane_live ? rbase + ((c0 + s + 1) % J) : lane;
-      x0 += lut[e0 * kRowStride + col0];
-      x1 += lut[e1 * kRowStride + col1];
+    for (int s = 0; s < J; ++s) {
+      const uint32_t off = __byte_perm(r.k[s >> 2], lane4, 0x5504u | (uint32_t(s & 3) << 4));
+      xa[s & 3] += *reinterpret_cast<const float*>(lut_bytes + off + 4 * s);
     }
     const bool valid = lane_live && (base + lane) < valid_in_page;
-    const float x = valid ? x0 + x1 : -INFINITY;
+    const float x = valid ? (xa[0] + xa[1]) + (xa[2] + xa[3]) : -INFINITY;
     const float xm = warp_max(x);                       // finite: slot 0 of the block is valid
     if (xm > m_w + kRescaleSlack) {                     // warp-uniform
       if (m_w != -INFINITY) {
         const float f = fast_exp2(m_w - xm);
+#pragma unroll 8
         for (int e = 0; e < kE; ++e) my_hist[e * kRowStride + lane] *= f;   // own column
         l_lane *= f;
       }
@@ -402,13 +402,15 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
       const float* pp = my_p + (lane / J) * J;
 #pragma unroll
       for (int i = 0; i < J; i += 2) {
-        const uint32_t ea = byte_of(r.v[i >> 2], i & 3);
-        const uint32_t eb = byte_of(r.v[(i + 1) >> 2], (i + 1) & 3);
+        // (e << 8 | lane*8) >> 1 = e*128 + lane*4: the byte offset of W[e][lane]
+        const uint32_t oa = __byte_perm(r.v[i >> 2], lane8, 0x5504u | (uint32_t(i & 3) << 4)) >> 1;
+        const uint32_t ob =
+            __byte_perm(r.v[(i + 1) >> 2], lane8, 0x5504u | (uint32_t((i + 1) & 3) << 4)) >> 1;
         const float2 pab = *reinterpret_cast<const float2*>(pp + i);
-        float* wa = my_hist + ea * kRowStride + lane;
-        float* wb = my_hist + eb * kRowStride + lane;
+        float* wa = reinterpret_cast<float*>(hist_bytes + oa);
+        float* wb = reinterpret_cast<float*>(hist_bytes + ob);
         const float va = *wa, vb = *wb;
-        const bool same = (ea == eb);
+        const bool same = (oa == ob);
         const float na = va + (same ? pab.x + pab.y : pab.x);
         const float nb = same ? na : vb + pab.y;
         *wa = na;
@@ -503,7 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
 }
 
 constexpr size_t decode_smem_bytes() {
-  return (static_cast<size_t>(kRegion) * (1 + kNW) + kNW * 32 + 2 * kNW) * sizeof(float);
+  return (static_cast<size_t>(kLutFloats) + static_cast<size_t>(kRegion) * kNW + kNW * 32 + 2 * kNW) *
+         sizeof(float);
 }
 static_assert(decode_smem_bytes() <= 227 * 1024, "decode kernel shared memory above 227 KB");
 
