@@ -44,6 +44,7 @@ constexpr int kLutRow = 64;             // LUT row: 64 columns, column k holds g
 constexpr int kLutFloats = kE * kLutRow;  // 64 KB
 constexpr int kStageRegions = 4;        // histogram regions 1..4 double as codebook staging
 constexpr int kWinChunk = 12;           // window tokens per warp per round of loads
+constexpr int kPrefetchPages = 8;       // pages a warp asks L2 to fetch ahead of its loads
 constexpr float kRescaleSlack = 8.0f;   // log2 units a new maximum may exceed m before rescaling
 
 struct DecodeParams {
@@ -192,13 +193,27 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   auto bt_entry = [&](int i) -> int { return (i < n_my_pages) ? bt[my_first + i * kNW] : -1; };
   int bt_cur = bt_entry(lane);
   int bt_nxt = bt_entry(32 + lane);
+  // L2 prefetch of this warp's first pages (lane l: page index l)
+  if (lane < kPrefetchPages && lane < n_my_pages && bt_cur >= 0 && bt_cur < p.n_pages)
+    prefetch_l2_bulk(pool_h + static_cast<int64_t>(bt_cur) * p.page_bytes,
+                     static_cast<uint32_t>(p.page_bytes));
+  const uint32_t bpp_magic = 0xFFFFFFFFu / static_cast<uint32_t>(bpp) + 1u;   // k / bpp = umulhi
   BlockRegs<J> ring[kDepth];
   auto issue = [&](int k, BlockRegs<J>& r) {
-    const int pi = k / bpp;
+    const int pi = static_cast<int>(__umulhi(static_cast<uint32_t>(k), bpp_magic));
+    const int blk = k - pi * bpp;
     if (pi >= i0 + 32) {                                // warp-uniform
       bt_cur = bt_nxt;
       i0 += 32;
       bt_nxt = bt_entry(i0 + 32 + lane);
+    }
+    if (blk == 0) {                                     // first block of a page: prefetch ahead
+      const int tgt = pi + kPrefetchPages;              // tgt - i0 < 64: inside cur or nxt
+      const int src = (tgt - i0 < 32) ? bt_cur : bt_nxt;
+      const int pf = __shfl_sync(0xffffffffu, src, (tgt - i0) & 31);
+      if (lane == 0 && tgt < n_my_pages && pf >= 0 && pf < p.n_pages)
+        prefetch_l2_bulk(pool_h + static_cast<int64_t>(pf) * p.page_bytes,
+                         static_cast<uint32_t>(p.page_bytes));
     }
     const int phys = __shfl_sync(0xffffffffu, bt_cur, pi - i0);
     r.ok = phys >= 0 && phys < p.n_pages;
@@ -210,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
       }
       return;
     }
-    load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, p.Pg, k % bpp,
+    load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, p.Pg, blk,
                   lane, r);
   };
 #pragma unroll
@@ -367,7 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1) vq_decode_kernel(const DecodePara
   float l_lane = 0.f;
 
   auto process = [&](int k, const BlockRegs<J>& r) {
-    const int pi = k / bpp, blk = k % bpp;
+    const int pi = static_cast<int>(__umulhi(static_cast<uint32_t>(k), bpp_magic));
+    const int blk = k - pi * bpp;
     const int pg = my_first + pi * kNW;
     const int valid_in_page = min(p.Pg, n_vq - pg * p.Pg);
     const int base = blk * LB;
