@@ -62,7 +62,7 @@ class _Layout(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libloopvq.so not built ({LIB_PATH}); run python -m sub_bit_vq_b200.build")
+        raise ImportError(f"libloopvq.so not built ({LIB_PATH}); run python sub_bit_vq_b200/build.py")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, I64, F, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
                         ctypes.c_size_t)

@@ -1,6 +1,6 @@
 """Build libloopvq.so in-tree for sm_100a with nvcc.
 
-``python -m sub_bit_vq_b200.build`` compiles every source under ``csrc/``
+``python sub_bit_vq_b200/build.py`` compiles every source under ``csrc/``
 into ``_build/`` and links ``sub_bit_vq_b200/libloopvq.so``. Objects are
 rebuilt when their source, a header, or the flags changed.
 """
