@@ -224,6 +224,39 @@ loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_s
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Decode attention that needs no workspace from the caller. The pages have
+ * no counterpart for this call; it exists for callers that cannot allocate
+ * device memory: code that receives only input and output pointers from a
+ * host program that owns all device memory (a plugin or callback interface),
+ * and code running under a fixed device-memory budget that forbids further
+ * allocations. Such callers cannot provide the scratch that
+ * loopvq_decode_attn takes.
+ *
+ * Computes exactly what loopvq_decode_attn computes, with the same
+ * arguments except `workspace`/`workspace_bytes`. The split-K scratch is a
+ * file-scope device array of LOOPVQ_STATIC_SCRATCH_BYTES bytes inside the
+ * library: every GPU that loads the library holds it until the process
+ * exits, and this call itself allocates and frees nothing. When
+ * loopvq_decode_workspace_bytes(cfg, batch, max_seq_len) exceeds
+ * LOOPVQ_STATIC_SCRATCH_BYTES the call returns LOOPVQ_ERR_WORKSPACE and
+ * launches nothing.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any
+ * stream capture. All calls on a device share the one array and it keeps
+ * the last call's contents (no initial contents are needed); calls whose
+ * kernels overlap on the GPU, e.g. on two streams without ordering, race
+ * on it and give undefined results.
+ */
+#define LOOPVQ_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+loopvq_status loopvq_decode_attn_noalloc(const loopvq_config* cfg, int layer, int loop_step,
+                                         int batch, int max_seq_len, const void* q,
+                                         const uint8_t* pool, const float* codebooks,
+                                         const int32_t* block_table, const int32_t* seq_lens,
+                                         const void* win_k, const void* win_v, float sm_scale,
+                                         int out_dtype, void* out, float* lse, void* stream);
+
+/*
  * Same-shape decode attention over a dense bf16 KV cache, the comparison
  * point for loopvq_decode_attn (the pages compare LoopVQ decode latency
  * with BF16 at 32K context: airadar.tv section "Raisons").

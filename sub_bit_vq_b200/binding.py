@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
     lib.loopvq_decode_attn.restype = I
     lib.loopvq_decode_attn.argtypes = [cfgp, I, I, I, I, P, P, P, P, P, P, P, F, I, P, P, P, SZ,
                                        P]
+    lib.loopvq_decode_attn_noalloc.restype = I
+    lib.loopvq_decode_attn_noalloc.argtypes = [cfgp, I, I, I, I, P, P, P, P, P, P, P, F, I, P, P, P]
     lib.loopvq_bf16_decode_workspace_bytes.restype = SZ
     lib.loopvq_bf16_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.loopvq_bf16_decode_attn.restype = I
@@ -88,7 +90,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 EXPORTED = ("loopvq_status_string", "loopvq_cache_layout", "loopvq_encode",
-            "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
+            "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
             "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn")
 
 
@@ -206,6 +208,31 @@ def loopvq_decode_attn(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.T
         float(sm_scale), odt, _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("loopvq_decode_attn", st)
+
+
+LOOPVQ_STATIC_SCRATCH_BYTES = 4 << 20
+
+
+def loopvq_decode_attn_noalloc(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.Tensor,
+                               pool: torch.Tensor, codebooks: torch.Tensor,
+                               block_table: torch.Tensor, seq_lens: torch.Tensor,
+                               win_k: torch.Tensor, win_v: torch.Tensor, out: torch.Tensor,
+                               max_seq_len: int, lse: torch.Tensor | None = None,
+                               sm_scale: float | None = None, stream=None) -> None:
+    """loopvq_decode_attn without a workspace argument: the split scratch is
+    the library's own static device array (for callers that cannot
+    allocate device memory). Calls that overlap on the GPU race on it."""
+    batch = q.shape[0]
+    if sm_scale is None:
+        sm_scale = cfg.head_dim ** -0.5
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    odt = LOOPVQ_DTYPE_F32 if out.dtype == torch.float32 else LOOPVQ_DTYPE_BF16
+    st = _lib.loopvq_decode_attn_noalloc(
+        cfg.c_ref(), layer, loop_step, batch, max_seq_len, _ptr(q), _ptr(pool), _ptr(codebooks),
+        _ptr(block_table), _ptr(seq_lens), _ptr(win_k), _ptr(win_v), float(sm_scale), odt,
+        _ptr(out), _ptr(lse), _stream(stream))
+    _check("loopvq_decode_attn_noalloc", st)
 
 
 def loopvq_bf16_decode_workspace_bytes(batch: int, n_q_heads: int, head_dim: int,
