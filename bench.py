@@ -45,6 +45,9 @@ def parse_args():
     ap.add_argument("--config", default="long32k")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the bf16-KV comparison and the prefill encode leg")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="fewer layers with the same per-call shape (small profiling case)")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     return ap.parse_args()
 
 
@@ -407,6 +410,8 @@ def main():
         args.warmup = 3
     from synthetic import SHAPES
     shape = SHAPES[args.config]
+    if args.layers is not None:
+        shape = shape.with_(n_layers=args.layers)
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -540,7 +545,7 @@ def main():
             "gpu_launches": wl.launches_per_step() * K,
             "clocks": clocks, "roofline": roofline}
 
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(shape)
     if rank == 0 and not args.no_extras:
         del wl
