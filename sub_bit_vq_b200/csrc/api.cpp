@@ -16,7 +16,6 @@ namespace {
 
 constexpr int kMaxCtas = 4096;    // upper bound on decode CTAs the planner targets
 constexpr int kCentroids = 256;   // 8-bit index
-constexpr int kMinSplitPages = 4; // fewest pages a context split should stream
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -168,10 +167,10 @@ loopvq_status loopvq_cache_layout(const loopvq_config* cfg, loopvq_layout* out) 
 size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int max_seq_len) {
   Geometry g;
   if (loopvq::make_geometry(cfg, &g) != LOOPVQ_OK || batch <= 0 || max_seq_len < 0) return 0;
-  const int pairs = batch * g.Hq;
-  const int pages = loopvq::pages_for(g, max_seq_len);
-  const int s = loopvq::max_decode_splits(pairs, pages);
-  return static_cast<size_t>(pairs) * s * (g.d + 2) * sizeof(float);
+  // one (m, l, o[d]) record per (pair, streaming CTA) segment: record slots
+  // pair + cta never collide, so pairs + CTAs slots suffice
+  const size_t slots = static_cast<size_t>(batch) * g.Hq + loopvq::kMaxStreamCtas;
+  return slots * (g.d + 2) * sizeof(float);
 }
 
 loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_idx, int kv,
@@ -233,16 +232,13 @@ loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_s
   loopvq_status err = LOOPVQ_OK;
   const int sms = loopvq::current_sm_count(&err);
   if (err != LOOPVQ_OK) return err;
-  const int pairs = batch * g.Hq;
-  int splits = (2 * sms + pairs - 1) / pairs;
-  const int by_pages = pages / loopvq::kMinSplitPages;
-  if (splits > by_pages) splits = by_pages;
-  const int smax = loopvq::max_decode_splits(pairs, pages);
-  if (splits > smax) splits = smax;
-  if (splits < 1) splits = 1;
+  // persistent streaming grid: one CTA per SM, never more CTAs than pages
+  const long long units_max = static_cast<long long>(batch) * g.Hq * pages;
+  int n_cta = sms < loopvq::kMaxStreamCtas ? sms : loopvq::kMaxStreamCtas;
+  if (units_max < n_cta) n_cta = static_cast<int>(units_max);
   loopvq::DecodeArgs a{&g,      layer,  loop_step,  batch,    max_seq_len, q,    pool,
                        codebooks, block_table, seq_lens, win_k, win_v,      sm_scale, out_dtype,
-                       out,     lse,    workspace,  splits,   stream};
+                       out,     lse,    workspace,  n_cta,    stream};
   return loopvq::launch_decode(a);
 }
 

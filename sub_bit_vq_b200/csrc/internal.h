@@ -20,8 +20,12 @@ struct Geometry {
 // Validates `cfg` and fills `geo`. Pure host code.
 loopvq_status make_geometry(const loopvq_config* cfg, Geometry* geo);
 
-// Largest number of context splits the decode planner may use.
+// Largest number of context splits the bf16-KV planner may use.
 int max_decode_splits(int pairs, int pages);
+
+// Most CTAs the persistent LoopVQ streaming kernel is launched with; the
+// decode workspace holds (pairs + kMaxStreamCtas) segment records.
+constexpr int kMaxStreamCtas = 1024;
 
 // Number of multiprocessors of the current device (cached per device).
 // Returns 0 and sets *err when the runtime fails.
@@ -43,7 +47,7 @@ struct DecodeArgs {
   void* out;
   float* lse;
   void* workspace;
-  int splits;
+  int n_cta;             // persistent streaming CTAs (0: nothing to stream)
   void* stream;
 };
 loopvq_status launch_decode(const DecodeArgs& a);

@@ -143,7 +143,10 @@ def test_workspace_bytes_formula():
     cfg = _cfg()
     # one (m, l, o[d]) float32 record per (sequence, query head, split)
     n = L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64)
-    assert n % (4 * (cfg.head_dim + 2) * 2 * cfg.n_q_heads) == 0
+    rec = 4 * (cfg.head_dim + 2)
+    assert n % rec == 0 and n >= rec * 2 * cfg.n_q_heads
+    # more sequences need more records
+    assert L.loopvq_decode_workspace_bytes(cfg, 4, 72 + 5 * 64) > n
     assert L.loopvq_decode_workspace_bytes(cfg, 0, 10) == 0
 
 
