@@ -54,6 +54,13 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
 }
 
+// 8-byte asynchronous global -> shared copy (cp.async, L1 allocating). Both
+// addresses must be 8-byte aligned.
+__device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
+
 // Asks L2 to fetch `bytes` (multiple of 16, 16-byte aligned address) from
 // global memory; no data is returned to the SM and nothing waits on it.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* gmem, uint32_t bytes) {

@@ -490,6 +490,314 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   }
 }
 
+// ---------------------------------------------------------------------------
+// Value path by explicit dequantisation (used when the loop-tau value
+// codebook slice fits in shared memory next to the key LUT).
+//
+// Same partition, segment walk, index stream and key pass as
+// vq_stream_kernel. The value slice is staged once per segment as
+// [E][C/CW][JP][CW] floats (JP = J rounded up so that the 16-byte reads of
+// the lanes of a warp fall on distinct bank groups). In the value pass a
+// lane = (replica, group j) accumulates o[j*c..j*c+c) += p * C_V[e][j] in
+// registers, one 16-byte shared read per slot: no read-modify-write, no
+// per-warp histogram, so the CTA runs kDqWarps warps and an online-softmax
+// rescale only touches registers.
+// ---------------------------------------------------------------------------
+
+constexpr int kDqWarps = 8;
+constexpr int kDqThreads = kDqWarps * 32;
+
+template <int J, int C>
+struct DqGeo {
+  static constexpr int CW = (C >= 4) ? 4 : C;          // floats per shared read
+  static constexpr int NH = C / CW;                    // reads per codeword slice
+  static constexpr int JP = (CW == 4) ? ((J + 7) / 8) * 8 : ((J + 15) / 16) * 16;
+  static constexpr int CV_FLOATS = kE * NH * JP * CW;  // [E][NH][JP][CW]
+  static constexpr int CK_FLOATS = J * kE * C;         // staged key slice [J][E][C]
+  static constexpr int STAGE_FLOATS = CV_FLOATS > CK_FLOATS ? CV_FLOATS : CK_FLOATS;
+  static constexpr int RSB = NH * JP * CW * 4;         // bytes per centroid row of the value slice
+};
+
+template <int J, int C>
+constexpr size_t dq_smem_bytes() {
+  return (static_cast<size_t>(kLutFloats) + DqGeo<J, C>::STAGE_FLOATS + kDqWarps * 32 * C +
+          kDqWarps * 64 + 2 * kDqWarps) *
+         sizeof(float);
+}
+
+template <int J, int C>
+constexpr bool dq_fits() {
+  return dq_smem_bytes<J, C>() <= 227 * 1024 && C % 2 == 0;
+}
+
+template <int J, int C>
+__global__ void __launch_bounds__(kDqThreads, 1) vq_stream_dq_kernel(const DecodeParams p) {
+  using T = Traits<J>;
+  using G = DqGeo<J, C>;
+  constexpr int d = J * C;
+  constexpr int LB = T::LB;
+  constexpr int NW = kDqWarps;
+
+  extern __shared__ __align__(16) float smem[];
+  float* lut = smem;                                   // [E][64]
+  float* stage = lut + kLutFloats;                     // key slice, then value slice
+  float* obuf = stage + G::STAGE_FLOATS;               // [NW][32][C] end-of-segment partials
+  float* pbuf = obuf + NW * 32 * C;                    // [NW][64]
+  float* wstat = pbuf + NW * 64;                       // [2*NW]
+  float* qs = obuf;                                    // q scratch (d floats) before the stream
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool lane_live = lane < LB;
+  const int vj = lane % J;                             // value pass: this lane's group
+  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+  const char* lut_bytes = reinterpret_cast<const char*>(lut);
+  const char* cv_bytes = reinterpret_cast<const char*>(stage) + vj * G::CW * 4;
+  float* my_p = pbuf + warp * 64;
+  const int bpp = p.Pg / LB;
+  const uint32_t bpp_magic = 0xFFFFFFFFu / static_cast<uint32_t>(bpp) + 1u;
+
+  int b_first;
+  long long pre_first;
+  const long long U = find_unit(p, -1, lane, &b_first, &pre_first);
+  const long long u_lo = U * blockIdx.x / p.n_cta;
+  const long long u_hi = U * (blockIdx.x + 1) / p.n_cta;
+  if (u_lo >= u_hi) return;
+  int b;
+  long long pre;
+  find_unit(p, u_lo, lane, &b, &pre);
+  int pages_b = seq_pages(p, b);
+  const long long off = u_lo - static_cast<long long>(p.Hq) * pre;
+  int hq = static_cast<int>(off / pages_b);
+  int pg_start = static_cast<int>(off % pages_b);
+  long long u = u_lo;
+
+  while (u < u_hi && b < p.B) {
+    const int seg_pages = static_cast<int>(min(static_cast<long long>(pages_b - pg_start), u_hi - u));
+    const int pg_lo = pg_start, pg_hi = pg_start + seg_pages;
+    const int hkv = hq / p.ratio;
+    const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
+    const int n_vq = max(0, N - p.W);
+    const float* cbk = p.cb_k + hkv * p.cb_stride_head;
+    const float* cbv = p.cb_v + hkv * p.cb_stride_head;
+    __syncthreads();                                   // previous segment done with shared memory
+
+    // ---- index ring prologue ------------------------------------------------
+    const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
+    const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages_per_seq;
+    const int my_first = pg_lo + warp;
+    const int n_my_pages = (pg_hi > my_first) ? (pg_hi - my_first + NW - 1) / NW : 0;
+    const int n_blocks = n_my_pages * bpp;
+    int i0 = 0;
+    auto bt_entry = [&](int i) -> int { return (i < n_my_pages) ? bt[my_first + i * NW] : -1; };
+    int bt_cur = bt_entry(lane);
+    int bt_nxt = bt_entry(32 + lane);
+    if (lane < kPrefetchPages && lane < n_my_pages && bt_cur >= 0 && bt_cur < p.n_pages)
+      prefetch_l2_bulk(pool_h + static_cast<int64_t>(bt_cur) * p.page_bytes,
+                       static_cast<uint32_t>(p.page_bytes));
+    BlockRegs<J> ring[kRing];
+    auto clear = [&](BlockRegs<J>& r) {
+      r.base = -1;
+#pragma unroll
+      for (int i = 0; i < T::NWORD; ++i) {
+        r.k[i] = 0u;
+        r.v[i] = 0u;
+      }
+    };
+    auto issue = [&](int k, BlockRegs<J>& r) {
+      if (k >= n_blocks) {
+        clear(r);
+        return;
+      }
+      const int pi = static_cast<int>(__umulhi(static_cast<uint32_t>(k), bpp_magic));
+      const int blk = k - pi * bpp;
+      if (pi >= i0 + 32) {
+        bt_cur = bt_nxt;
+        i0 += 32;
+        bt_nxt = bt_entry(i0 + 32 + lane);
+      }
+      if (blk == 0) {
+        const int tgt = pi + kPrefetchPages;
+        const int src = (tgt - i0 < 32) ? bt_cur : bt_nxt;
+        const int pf = __shfl_sync(0xffffffffu, src, (tgt - i0) & 31);
+        if (lane == 0 && tgt < n_my_pages && pf >= 0 && pf < p.n_pages)
+          prefetch_l2_bulk(pool_h + static_cast<int64_t>(pf) * p.page_bytes,
+                           static_cast<uint32_t>(p.page_bytes));
+      }
+      const int phys = __shfl_sync(0xffffffffu, bt_cur, pi - i0);
+      const int pg = my_first + pi * NW;
+      r.valid = min(p.Pg, n_vq - pg * p.Pg);
+      r.base = blk * LB;
+      if (phys < 0 || phys >= p.n_pages || r.base >= r.valid) {
+        clear(r);
+        return;
+      }
+      load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, p.Pg, blk,
+                    lane, r);
+    };
+#pragma unroll
+    for (int u2 = 0; u2 < kRing; ++u2) issue(u2, ring[u2]);
+
+    // ---- key LUT from the staged key slice ---------------------------------
+    stage_async<kDqThreads>(stage, cbk, G::CK_FLOATS, tid);
+    const uint16_t* qp = p.q + (static_cast<size_t>(b) * p.Hq + hq) * d;
+    for (int i = tid; i < d; i += kDqThreads) qs[i] = bf16_bits_to_float(qp[i]) * p.scale_log2;
+    cp_async_wait_all();
+    __syncthreads();
+    for (int item = warp; item < (kE / 32) * J; item += NW) {
+      const int tile = item / J, s = item % J;
+      const int e = tile * 32 + lane;
+      const int j = (lane + s) % J;
+      const float v = dot_c<C>(qs + j * C, stage + (static_cast<size_t>(j) * kE + e) * C);
+#pragma unroll
+      for (int k = j; k < kLutRow; k += J) lut[e * kLutRow + k] = v;
+    }
+    __syncthreads();                                   // LUT done; key slice no longer read
+    // ---- value slice [E][NH][JP][CW] ----------------------------------------
+    for (int idx = tid; idx < J * kE * G::NH; idx += kDqThreads) {
+      const int j = idx / (kE * G::NH), rem = idx % (kE * G::NH);
+      const int e = rem / G::NH, h = rem % G::NH;
+      const float* src = cbv + (static_cast<size_t>(j) * kE + e) * C + h * G::CW;
+      float* dst = stage + ((e * G::NH + h) * G::JP + j) * G::CW;
+      if constexpr (G::CW == 4)
+        cp_async16(dst, src);
+      else
+        cp_async8(dst, src);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- stream -------------------------------------------------------------
+    float m_w = -INFINITY;
+    float l_lane = 0.f;
+    float o[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) o[c] = 0.f;
+
+    auto key_scores = [&](const BlockRegs<J>& r) -> float {
+      float xa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < J; ++s) {
+        const uint32_t ob = __byte_perm(r.k[s >> 2], lane4, 0x5504u | (uint32_t(s & 3) << 4));
+        xa[s & 3] += *reinterpret_cast<const float*>(lut_bytes + ob + 4 * s);
+      }
+      const bool valid = r.base >= 0 && lane_live && (r.base + lane) < r.valid;
+      return valid ? (xa[0] + xa[1]) + (xa[2] + xa[3]) : -INFINITY;
+    };
+    auto value_pass = [&](const BlockRegs<J>& r, const float* pp) {
+      if (r.base < 0 || !lane_live) return;
+      pp += (lane / J) * J;
+#pragma unroll
+      for (int i = 0; i < J; i += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(pp + i);
+        const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t e = byte_of(r.v[i >> 2], k);
+          const char* row = cv_bytes + e * G::RSB;
+#pragma unroll
+          for (int h = 0; h < G::NH; ++h) {
+            if constexpr (G::CW == 4) {
+              const float4 cw = *reinterpret_cast<const float4*>(row + h * G::JP * 16);
+              o[4 * h] = fmaf(pv[k], cw.x, o[4 * h]);
+              o[4 * h + 1] = fmaf(pv[k], cw.y, o[4 * h + 1]);
+              o[4 * h + 2] = fmaf(pv[k], cw.z, o[4 * h + 2]);
+              o[4 * h + 3] = fmaf(pv[k], cw.w, o[4 * h + 3]);
+            } else {
+              const float2 cw = *reinterpret_cast<const float2*>(row + h * G::JP * 8);
+              o[2 * h] = fmaf(pv[k], cw.x, o[2 * h]);
+              o[2 * h + 1] = fmaf(pv[k], cw.y, o[2 * h + 1]);
+            }
+          }
+        }
+      }
+    };
+    auto process_pair = [&](const BlockRegs<J>& ra, const BlockRegs<J>& rb) {
+      const float xa = key_scores(ra);
+      const float xb = key_scores(rb);
+      const float xm = warp_max(fmaxf(xa, xb));
+      if (xm == -INFINITY) return;
+      if (xm > m_w + kRescaleSlack) {
+        if (m_w != -INFINITY) {
+          const float f = fast_exp2(m_w - xm);
+#pragma unroll
+          for (int c = 0; c < C; ++c) o[c] *= f;
+          l_lane *= f;
+        }
+        m_w = xm;
+      }
+      const float pa = (xa == -INFINITY) ? 0.f : fast_exp2(xa - m_w);
+      const float pb = (xb == -INFINITY) ? 0.f : fast_exp2(xb - m_w);
+      l_lane += pa + pb;
+      my_p[lane] = pa;
+      my_p[32 + lane] = pb;
+      __syncwarp();
+      value_pass(ra, my_p);
+      value_pass(rb, my_p + 32);
+      __syncwarp();                                    // my_p is rewritten by the next step
+    };
+
+    for (int k0 = 0; k0 < n_blocks; k0 += kRing) {
+      process_pair(ring[0], ring[1]);
+      issue(k0 + kRing, ring[0]);
+      issue(k0 + kRing + 1, ring[1]);
+      if (k0 + 2 >= n_blocks) break;
+      process_pair(ring[2], ring[3]);
+      issue(k0 + kRing + 2, ring[2]);
+      issue(k0 + kRing + 3, ring[3]);
+    }
+    const float l_w = warp_sum(l_lane);
+    if (lane == 0) {
+      wstat[warp] = m_w;
+      wstat[NW + warp] = l_w;
+    }
+#pragma unroll
+    for (int c = 0; c < C; ++c) obuf[(warp * 32 + lane) * C + c] = lane_live ? o[c] : 0.f;
+    __syncthreads();
+
+    // ---- merge warps into the segment record --------------------------------
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wstat[w]);
+    float* rec = p.records + static_cast<size_t>(b * p.Hq + hq + blockIdx.x) * (d + 2);
+    if (M == -INFINITY) {
+      for (int i = tid; i < d + 2; i += kDqThreads) rec[i] = (i == 0) ? -INFINITY : 0.f;
+    } else {
+      float L = 0.f;
+      float f[NW];
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        f[w] = (wstat[w] == -INFINITY) ? 0.f : fast_exp2(wstat[w] - M);
+        L += f[w] * wstat[NW + w];
+      }
+      for (int oi = tid; oi < d; oi += kDqThreads) {
+        const int j = oi / C, c = oi % C;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          float s = 0.f;
+#pragma unroll
+          for (int r = 0; r < T::R; ++r) s += obuf[(w * 32 + r * J + j) * C + c];
+          acc = fmaf(f[w], s, acc);
+        }
+        rec[2 + oi] = acc;
+      }
+      if (tid == 0) {
+        rec[0] = M;
+        rec[1] = L;
+      }
+    }
+
+    u += seg_pages;
+    pg_start = 0;
+    if (++hq == p.Hq) {
+      hq = 0;
+      do {
+        ++b;
+      } while (b < p.B && u < u_hi && (pages_b = seq_pages(p, b)) == 0);
+    }
+  }
+}
+
 // One CTA per (sequence, query head): the bf16 window partial, merged with
 // the pair's segment records into out and lse.
 template <int D>
@@ -664,10 +972,31 @@ constexpr size_t stream_smem_bytes() {
 }
 static_assert(stream_smem_bytes() <= 227 * 1024, "stream kernel shared memory above 227 KB");
 
+template <typename K>
+loopvq_status set_smem(K kernel, size_t smem, std::atomic<uint64_t>& configured) {
+  // The attribute belongs to (function, device); remember which devices have it.
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit == 0 || !(configured.load(std::memory_order_relaxed) & bit)) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return LOOPVQ_ERR_CUDA;
+    configured.fetch_or(bit, std::memory_order_relaxed);
+  }
+  return LOOPVQ_OK;
+}
+
 template <int J, int C>
 loopvq_status launch_vq(const DecodeParams& p, cudaStream_t st, bool run_stream) {
   constexpr int d = J * C;
-  if (run_stream) {
+  if (run_stream && dq_fits<J, C>()) {
+    static std::atomic<uint64_t> configured{0};
+    const size_t smem = dq_smem_bytes<J, C>();
+    if (set_smem(vq_stream_dq_kernel<J, C>, smem, configured) != LOOPVQ_OK) return LOOPVQ_ERR_CUDA;
+    vq_stream_dq_kernel<J, C><<<p.n_cta, kDqThreads, smem, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return LOOPVQ_ERR_CUDA;
+  } else if (run_stream) {
     const size_t smem = stream_smem_bytes();
     // The attribute belongs to (function, device); remember which devices have it.
     static std::atomic<uint64_t> configured{0};
