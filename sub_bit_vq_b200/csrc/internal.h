@@ -23,9 +23,10 @@ loopvq_status make_geometry(const loopvq_config* cfg, Geometry* geo);
 // Largest number of context splits the bf16-KV planner may use.
 int max_decode_splits(int pairs, int pages);
 
-// Most CTAs the persistent LoopVQ streaming kernel is launched with; the
-// decode workspace holds (pairs + kMaxStreamCtas) segment records.
-constexpr int kMaxStreamCtas = 1024;
+// Most CTAs the persistent LoopVQ streaming kernel is launched with (one per
+// SM up to this many); the decode workspace holds (pairs + kMaxStreamCtas)
+// segment records of 4 + 256*J floats.
+constexpr int kMaxStreamCtas = 256;
 
 // Number of multiprocessors of the current device (cached per device).
 // Returns 0 and sets *err when the runtime fails.

@@ -141,9 +141,10 @@ def test_encode_rejects_before_launch():
 
 def test_workspace_bytes_formula():
     cfg = _cfg()
-    # one (m, l, o[d]) float32 record per (sequence, query head, split)
+    # one record (m, l, 2 spare, value histogram [256][J]) of float32 per
+    # (sequence, query head, split)
     n = L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64)
-    rec = 4 * (cfg.head_dim + 2)
+    rec = 4 * (4 + 256 * (cfg.head_dim // cfg.chan_group))
     assert n % rec == 0 and n >= rec * 2 * cfg.n_q_heads
     # more sequences need more records
     assert L.loopvq_decode_workspace_bytes(cfg, 4, 72 + 5 * 64) > n
