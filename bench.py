@@ -525,7 +525,7 @@ def main():
                     "sub_bit_vq_b200/csrc/decode.cu", "vq_decode_long32k"),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)" if
                 peak_src == "measured" else "fallback 6650 GB/s",
-                "kernel": "vq_decode_kernel + merge_kernel (per-call events)",
+                "kernel": "vq_stream_kernel + vq_finish_kernel (per-call events)",
                 "algorithmic_bytes_per_launch": alg, "avg_launch_us": avg_call_us,
                 "frac_of_8tbs": achieved / 8000.0}
 

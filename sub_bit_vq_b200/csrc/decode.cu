@@ -2,17 +2,17 @@
 //
 // Two kernels per call.
 //
-// vq_stream_kernel: a persistent grid (at most one CTA per SM, eight warps)
+// vq_stream_kernel: a persistent grid (at most one CTA per SM, twelve warps)
 // over the quantised tokens of every (sequence, query head) pair. All pages
 // of all pairs form one list and CTA c takes the contiguous range
 // [U*c/n, U*(c+1)/n) of it, so every CTA streams the same number of pages and
 // touches one or a few pairs ("segments"). Per segment:
-//   1. The warps request their first index blocks (a register ring) and
-//      build the key lookup table LUT[e][col] = s*log2(e) * q_j . C_K[j][e][tau]
-//      (column col holds group j = col % J) from the key codebook slice read
-//      through L2. The segment that holds the pair's first page also scores
-//      the bf16 window tokens (prefix + recent) into a window partial.
-//   2. Streaming. Warp w takes pages w, w+8, ...; a block is LB token slots
+//   1. The key codebook slice of the pair's kv-head and loop step is staged
+//      into the (empty) histogram windows with cp.async while the warps
+//      request their first index blocks (a register ring); the key lookup
+//      table LUT[e][col] = s*log2(e) * q_j . C_K[j][e][tau] (column col holds
+//      group j = col % J) is built from it and the windows are zeroed.
+//   2. Streaming. Warp w takes pages w, w+12, ...; a block is LB token slots
 //      (LB = floor(32/J)*J), two blocks per round. Key pass: lane = slot;
 //      byte s of the slot's rotated row is group (lane+s) % J, held by LUT
 //      column (lane+s) % LB. Value pass: the weights p = 2^(x - m) are added
@@ -20,27 +20,27 @@
 //      `lane`, rows come from the group-major value bytes, four slots at a
 //      time; a weight whose row repeats later among the four is folded into
 //      that later update, so the last store of a row carries all of them.
-//      Two warps share one histogram and take turns through an mbarrier
-//      hand-off: one computes key scores while the other updates the
-//      histogram. The pair keeps one running maximum m, raised only when a
-//      vote finds a score above m + kRescaleSlack.
-//   3. The four histograms are merged and contracted with the value codebook
-//      slice read through L2, o_j = sum_e W[e][j] C_V[j][e][tau]; the window
-//      partial is folded in and the segment writes (m, l, o[d]) to record
-//      slot (pair + cta).
+//      Three warps (w, w+4, w+8: one scheduler) share a histogram and take
+//      turns through bounded mbarrier waits; a warp computes its key scores
+//      and weights before its turn and only the histogram updates inside it.
+//      Each histogram keeps one running maximum m, raised only when a vote
+//      finds a score above m + kRescaleSlack.
+//   3. The four histograms are merged into the segment record
+//      (m, l, W[E][J]) at slot (pair + cta).
 //
-// vq_finish_kernel: one CTA per pair merges the pair's segment records
-// (log-sum-exp merge) into out and lse. A pair without quantised pages has
-// no segment; its window partial is computed there.
+// vq_finish_kernel: one CTA per pair scores the bf16 window tokens (prefix +
+// recent), merges the pair's segment histograms with log-sum-exp weights,
+// contracts the merged histogram with the value codebook slice,
+// o_j = sum_e W[e][j] C_V[j][e][tau], and writes out and lse.
 //
 // The hot loops address shared memory by absolute shared-window address, so
 // that one byte permute of an index word gives a complete address: the
 // histograms occupy the 64 KB-aligned windows [0x10000, 0x30000) (row e at
-// byte e*256 of its window, two histograms per window), the LUT the window
-// [0x8000, 0x10000) with 128-byte rows, and scratch starts at 0x30000. The
-// dynamic allocation starts at a small base (the CTA's reserved bytes) and is
-// sized to cover all of them; a CTA whose base leaves no room writes NaN
-// records instead of running.
+// byte e*256 of its window, two histograms per window) and the LUT the
+// window [0x8000, 0x10000) with 128-byte rows. The dynamic allocation starts
+// at a small base (the CTA's reserved bytes) and is sized to cover both; a
+// CTA whose base leaves no room below the LUT writes NaN records instead of
+// running.
 
 #include <math.h>
 
@@ -235,8 +235,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
 // the phase completes or kSuspendNs pass); gives up (false) after kSpinLimit
 // tries instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
-  for (int i = 0; i < kSpinLimit; ++i)
+  for (int i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(a, parity)) return true;
+    __nanosleep(64);                                   // leave the issue slots to the working warps
+  }
   return false;
 }
 
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   constexpr int JC = (J * kE * C * 4 <= static_cast<int>(kHistEnd - kHistAbs))
                          ? J : static_cast<int>(kHistEnd - kHistAbs) / (kE * C * 4);
   static_assert(J % JC == 0, "staging chunks tile the groups");
-  static_assert(d <= kNW * 64, "q fits the weight buffer");
+  static_assert(d <= kNW * 64 && d <= kThreads, "q fits the weight buffer");
 
   extern __shared__ __align__(16) unsigned char smem_u8[];
   const uint32_t sbase = smem_addr(smem_u8);
@@ -471,6 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       const float* cbk = p.cb_k + hkv * p.cb_stride_head;
       const uint16_t* qp = p.q + (static_cast<size_t>(b) * p.Hq + hq) * d;
       __syncthreads();                                 // previous segment done with LUT and histograms
+      // the first chunk of the key slice goes out before anything that waits
+      for (int i = tid * 4; i < JC * kE * C; i += kThreads * 4) cp_async16(stage + i, cbk + i);
+      const float qv = (tid < d) ? bf16_bits_to_float(qp[tid]) * p.scale_log2 : 0.f;
 
       // ---- index ring prologue ----------------------------------------------
       const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
@@ -530,12 +535,14 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       for (int k = 0; k < kRing; ++k) issue(k, ring[k]);
 
       // ---- key LUT from the key slice staged in the histogram windows ----------
-      for (int i = tid; i < d; i += kThreads) qs[i] = bf16_bits_to_float(qp[i]) * p.scale_log2;
+      if (tid < d) qs[tid] = qv;
 #pragma unroll 1
       for (int j0 = 0; j0 < J; j0 += JC) {
-        if (j0 > 0) __syncthreads();                   // previous chunk consumed
-        const float* src = cbk + static_cast<size_t>(j0) * kE * C;
-        for (int i = tid * 4; i < JC * kE * C; i += kThreads * 4) cp_async16(stage + i, src + i);
+        if (j0 > 0) {
+          __syncthreads();                             // previous chunk consumed
+          const float* src = cbk + static_cast<size_t>(j0) * kE * C;
+          for (int i = tid * 4; i < JC * kE * C; i += kThreads * 4) cp_async16(stage + i, src + i);
+        }
         cp_async_wait_all();
         __syncthreads();
         // item = (tile of 32 rows, step): lane -> row tile*32 + lane, group
@@ -591,19 +598,30 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           sts_h(a3, o3 + q3);
         }
       };
-      // One round: key scores outside the turn, weights and histogram inside.
+      // One round: key scores and (against the maximum this warp saw last)
+      // weights outside the turn, the histogram updates inside.
       auto round = [&](const BlockRegs<J>& ra, const BlockRegs<J>& rb) {
         const float xa = key_scores(ra);
         const float xb = key_scores(rb);
+        const float xl = fmaxf(xa, xb);
+        const bool spec = m_seen != -INFINITY &&
+                          __all_sync(0xffffffffu, !(xl > m_seen + kRescaleSlack));
+        float pa = 0.f, pb = 0.f;
+        if (spec) {                                    // warp-uniform
+          pa = fast_exp2(xa - m_seen);
+          pb = fast_exp2(xb - m_seen);
+          my_p[lane] = pa;
+          my_p[32 + lane] = pb;
+        }
         if (!wait_failed && !mbar_wait(bar_wait, rnd & 1u)) wait_failed = true;
         ++rnd;
         float m = hm[hidx];
-        if (m != m_seen) {                             // the partner raised the maximum
+        const bool keep = spec && m == m_seen;         // warp-uniform
+        if (m != m_seen) {                             // another warp raised the maximum
           if (m_seen != -INFINITY) l_lane *= fast_exp2(m_seen - m);
           m_seen = m;
         }
-        const float xl = fmaxf(xa, xb);
-        if (__any_sync(0xffffffffu, xl > m + kRescaleSlack)) {   // warp-uniform, rare
+        if (!keep && __any_sync(0xffffffffu, xl > m + kRescaleSlack)) {   // warp-uniform, rare
           const float xm = warp_max(xl);
           if (m != -INFINITY) {
             const float f = fast_exp2(m - xm);
@@ -620,11 +638,13 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           if (lane == 0) hm[hidx] = xm;
         }
         if (m != -INFINITY) {                          // warp-uniform
-          const float pa = fast_exp2(xa - m);          // 0 for xa = -inf
-          const float pb = fast_exp2(xb - m);
+          if (!keep) {
+            pa = fast_exp2(xa - m);                    // 0 for xa = -inf
+            pb = fast_exp2(xb - m);
+            my_p[lane] = pa;
+            my_p[32 + lane] = pb;
+          }
           l_lane += pa + pb;
-          my_p[lane] = pa;
-          my_p[32 + lane] = pb;
           __syncwarp();
           value_pass(ra, my_p);
           value_pass(rb, my_p + 32);
@@ -669,13 +689,13 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
 #pragma unroll
         for (int h = 0; h < kNHist; ++h) fh[h] = (hm[h] == -INFINITY) ? 0.f : fast_exp2(hm[h] - Mh);
         // lane = column, rows warp + kNW*k; replicas of a group are summed
+        const float* hist = stage;                     // the histogram windows as floats
         for (int e = warp; e < kE; e += kNW) {
           float v = 0.f;
           if (lane_live) {
 #pragma unroll
             for (int h = 0; h < kNHist; ++h)
-              v = fmaf(fh[h], lds_h(((1u + (h >> 1)) << 16) | (static_cast<uint32_t>(e) << 8) |
-                                    static_cast<uint32_t>((h & 1) * 128 + lane * 4)), v);
+              v = fmaf(fh[h], hist[(h >> 1) * 16384 + e * 64 + (h & 1) * 32 + lane], v);
           }
 #pragma unroll
           for (int o = (T::R / 2) * J; o >= J; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
@@ -776,13 +796,29 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
   bool any_hist = false;
   for (int c = c_first; c <= c_last; ++c) any_hist |= fc[c - c_first] != 0.f;
   if (any_hist) {                                      // CTA-uniform
-    for (int i = tid; i < kE * J; i += kFinishThreads) {
-      float h = 0.f;
-      for (int c = c_first; c <= c_last; ++c) {
-        const float f = fc[c - c_first];
-        if (f != 0.f) h = fmaf(f, p.records[static_cast<size_t>(pair + c) * RS + 4 + i], h);
+    // every thread owns the same PER words of each record: a record's words
+    // are requested together, one record after another
+    constexpr int PER = (kE * J + kFinishThreads - 1) / kFinishThreads;
+    float hacc[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) hacc[k] = 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+      const float f = fc[c - c_first];
+      if (f == 0.f) continue;                          // CTA-uniform
+      const float* r = p.records + static_cast<size_t>(pair + c) * RS + 4;
+      float v[PER];
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int i = tid + k * kFinishThreads;
+        v[k] = (i < kE * J) ? __ldcg(r + i) : 0.f;
       }
-      hs[(i / J) * JP + i % J] = h;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) hacc[k] = fmaf(f, v[k], hacc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int i = tid + k * kFinishThreads;
+      if (i < kE * J) hs[(i / J) * JP + i % J] = hacc[k];
     }
     __syncthreads();
     // warp -> groups j = warp, warp + NW, ..; lane -> rows lane + 32*i
