@@ -56,6 +56,8 @@ def parse_args():
 # --------------------------------------------------------------------------
 
 def dist_init(n_gpus: int):
+    """One process per GPU (torchrun env). NCCL between GPUs; gloo when no
+    GPU is visible (the host-side logic is exercised that way on CPU)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -63,9 +65,12 @@ def dist_init(n_gpus: int):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=300)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
@@ -82,9 +87,18 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(elapsed_ms: float, steps: int, n_loops: int, world: int):
+    """µs per loop step of the whole job and ms per bench step. Every rank
+    runs `steps` steps of `n_loops` loop steps on its own replica (weak
+    scaling); elapsed_ms is the max over ranks."""
+    loop_steps = steps * n_loops * world
+    return elapsed_ms * 1e3 / loop_steps, elapsed_ms / steps
 
 
 # --------------------------------------------------------------------------
@@ -415,7 +429,8 @@ def main():
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
-        if rank != 0:
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:                                  # rank 0 alone times the oracle
             return 0
         for _ in range(args.warmup):
             cpu_baseline(shape, budget_s=0.5)
@@ -425,7 +440,7 @@ def main():
         rec = dict(vals[-1])
         rec["value"] = v
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "µs/loop-step",
-                "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": v * shape.n_loops / 1e3, "higher_is_better": False,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": shape.name, "batch": shape.batch, "context": shape.context,
@@ -474,8 +489,7 @@ def main():
     avg_call_us = sum(call_us) / len(call_us)
 
     loop_steps = K * shape.n_loops * world
-    value = elapsed_ms * 1e3 / loop_steps
-    ms_per_step = elapsed_ms / K
+    value, ms_per_step = whole_job_value(elapsed_ms, K, shape.n_loops, world)
 
     # end to end through the public API with host buffers: per step the
     # queries, the new token's K/V rows and the evicted token come from
