@@ -16,6 +16,8 @@ namespace loopvq {
 namespace {
 
 constexpr int kEncThreads = 128;
+constexpr int kEncWarpThreads = 256;    // small batches: one CTA per (group, head), a warp per token
+constexpr int kEncWarpMaxTokens = 64;   // batches up to this size take the warp form
 
 struct EncodeParams {
   const uint16_t* x;            // bf16 bits
@@ -30,6 +32,104 @@ struct EncodeParams {
   int64_t n_slots;              // n_pages * Pg
   int n_tokens, d, Pg, J, LB, GR, kv;
 };
+
+// Writes index `e` of (slot, group j, head h) to its byte in the pool.
+__device__ __forceinline__ void store_index(const EncodeParams& p, int64_t slot, int j, int h, int e) {
+  const int64_t page = slot / p.Pg;
+  const int sl = static_cast<int>(slot % p.Pg);
+  int64_t off;
+  if (p.kv == 0) {                          // K plane: rotated slot rows
+    const int blk = sl / p.LB, rot = sl % p.LB;
+    int pos = j - rot % p.J;
+    if (pos < 0) pos += p.J;
+    off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR + rot * p.GR +
+          pos % p.GR;
+  } else {                                  // V plane: group-major
+    off = static_cast<int64_t>(j) * p.Pg + sl;
+  }
+  p.pool[h * p.pool_stride_head + page * p.page_bytes + p.kv * p.plane_bytes + off] =
+      static_cast<uint8_t>(e);
+}
+
+// Loads token n's sub-vector of (group j, head h) and its weights (1 when
+// no weights are given).
+template <int C, int G>
+__device__ __forceinline__ void load_subvector(const EncodeParams& p, int n, int j, int h,
+                                               float (&s)[C * G], float (&w)[C * G]) {
+#pragma unroll
+  for (int tau = 0; tau < G; ++tau) {
+    const uint16_t* xr = p.x + tau * p.x_loop_stride + n * p.x_token_stride +
+                         static_cast<int64_t>(h) * p.d + j * C;
+#pragma unroll
+    for (int ch = 0; ch < C; ++ch) s[tau * C + ch] = bf16_bits_to_float(xr[ch]);
+    if (p.w != nullptr) {
+      const float* wr = p.w + tau * p.w_loop_stride + n * p.w_token_stride +
+                        static_cast<int64_t>(h) * p.d + j * C;
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = wr[ch];
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = 1.f;
+    }
+  }
+}
+
+// Small batches (the tokens leaving the recent window at each decode step):
+// one CTA per (group j, head h) stages the codebook of (j, h) once as
+// [tau][E][c]; each warp takes tokens warp, warp+8, .., the lanes scan
+// centroids lane, lane+32, .. with the same float32 weighted distance and
+// term order as encode_kernel, and a shuffle argmin keeps the smallest
+// index among equal distances.
+template <int C, int G>
+__global__ void __launch_bounds__(kEncWarpThreads) encode_warp_kernel(const EncodeParams p) {
+  constexpr int D = C * G;
+  __shared__ __align__(16) float cbs[G * kE * C];
+  const int j = blockIdx.x, h = blockIdx.y;
+  const float* cb = p.cb + h * p.cb_stride_head + static_cast<int64_t>(j) * kE * C;
+  for (int i = threadIdx.x * 4; i < G * kE * C; i += kEncWarpThreads * 4) {
+    const int tau = i / (kE * C), r = i % (kE * C);
+    cp_async16(cbs + i, cb + tau * p.cb_stride_loop + r);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int n = warp; n < p.n_tokens; n += kEncWarpThreads / 32) {
+    const int64_t slot = p.slot_mapping[n];
+    if (slot < 0 || slot >= p.n_slots) continue;   // warp-uniform
+    float s[D], w[D];
+    load_subvector<C, G>(p, n, j, h, s, w);
+    float best = INFINITY;
+    int best_e = 0;
+#pragma unroll 2
+    for (int k = 0; k < kE / 32; ++k) {
+      const int e = 32 * k + lane;
+      float dist = 0.f;
+#pragma unroll
+      for (int tau = 0; tau < G; ++tau) {
+        const float* cw = cbs + (tau * kE + e) * C;
+#pragma unroll
+        for (int ch = 0; ch < C; ++ch) {
+          const float df = s[tau * C + ch] - cw[ch];
+          dist = fmaf(w[tau * C + ch] * df, df, dist);
+        }
+      }
+      if (dist < best) {
+        best = dist;
+        best_e = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float od = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
+      if (od < best || (od == best && oe < best_e)) {
+        best = od;
+        best_e = oe;
+      }
+    }
+    if (lane == 0) store_index(p, slot, j, h, best_e);
+  }
+}
 
 template <int C, int G>
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams p) {
@@ -48,22 +148,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
   if (slot < 0 || slot >= p.n_slots) return;
 
   float s[D], w[D];
-#pragma unroll
-  for (int tau = 0; tau < G; ++tau) {
-    const uint16_t* xr = p.x + tau * p.x_loop_stride + n * p.x_token_stride +
-                         static_cast<int64_t>(h) * p.d + j * C;
-#pragma unroll
-    for (int ch = 0; ch < C; ++ch) s[tau * C + ch] = bf16_bits_to_float(xr[ch]);
-    if (p.w != nullptr) {
-      const float* wr = p.w + tau * p.w_loop_stride + n * p.w_token_stride +
-                        static_cast<int64_t>(h) * p.d + j * C;
-#pragma unroll
-      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = wr[ch];
-    } else {
-#pragma unroll
-      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = 1.f;
-    }
-  }
+  load_subvector<C, G>(p, n, j, h, s, w);
 
   float best = INFINITY;
   int best_e = 0;
@@ -87,24 +172,15 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
     }
   }
 
-  const int64_t page = slot / p.Pg;
-  const int sl = static_cast<int>(slot % p.Pg);
-  int64_t off;
-  if (p.kv == 0) {                          // K plane: rotated slot rows
-    const int blk = sl / p.LB, rot = sl % p.LB;
-    int pos = j - rot % p.J;
-    if (pos < 0) pos += p.J;
-    off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR + rot * p.GR +
-          pos % p.GR;
-  } else {                                  // V plane: group-major
-    off = static_cast<int64_t>(j) * p.Pg + sl;
-  }
-  p.pool[h * p.pool_stride_head + page * p.page_bytes + p.kv * p.plane_bytes + off] =
-      static_cast<uint8_t>(best_e);
+  store_index(p, slot, j, h, best_e);
 }
 
 template <int C, int G>
 loopvq_status launch_enc(const EncodeParams& p, int J, int H, cudaStream_t st) {
+  if (p.n_tokens <= kEncWarpMaxTokens) {
+    encode_warp_kernel<C, G><<<dim3(J, H), kEncWarpThreads, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+  }
   const dim3 grid((p.n_tokens + kEncThreads - 1) / kEncThreads, J, H);
   encode_kernel<C, G><<<grid, kEncThreads, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;

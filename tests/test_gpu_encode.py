@@ -163,3 +163,49 @@ def test_zero_tokens_is_a_noop():
                     torch.zeros(1, dtype=torch.int64, device="cuda"), pool)
     torch.cuda.synchronize()
     assert not pool.any()
+
+
+@pytest.mark.parametrize("n", [1, 8, 37, 64])
+def test_small_batches_weighted_with_skips(n):
+    # batches of at most 64 tokens (the window eviction at each decode step)
+    # take the warp-per-token kernel
+    s = W128
+    layer, gamma, kv, n_pages = 1, 0, 1, 3
+    x = loop_group_kv(s, layer, gamma, kv, n)
+    w = weights(s, n, True, layer, gamma, kv)
+    cb = random_codebooks(s, 2, 12)
+    slots = _slots(n, n_pages, s.page_tokens, 13, skip_every=5 if n > 5 else 0)
+    pool = _run(s, 2, layer, gamma, kv, x, w, cb, slots, n_pages)
+    _, dist = O.encode_group_ref(x.double().numpy(), cb[layer, :, gamma, kv].double().numpy(),
+                                 w.double().numpy())
+    keep = slots >= 0
+    check_indices(_gpu_indices(pool, s, layer, gamma, kv, slots)[keep], dist[keep])
+
+
+def test_small_batch_j12_and_ties():
+    s = J12
+    n, n_pages = 24, 2
+    x = loop_group_kv(s, 0, 0, 0, n)
+    cb = random_codebooks(s, 1, 14)
+    slots = _slots(n, n_pages, s.page_tokens, 15)
+    pool = _run(s, 1, 0, 0, 0, x, None, cb, slots, n_pages)
+    _, dist = O.encode_group_ref(x.double().numpy(), cb[0, :, 0, 0].double().numpy())
+    check_indices(_gpu_indices(pool, s, 0, 0, 0, slots), dist)
+    # exact codewords with a duplicated codeword: the smaller index wins
+    t = W128.with_(n_kv_heads=1, n_q_heads=1)
+    g, J, c, E = t.loop_group, t.J, t.chan_group, 256
+    gen = torch.Generator().manual_seed(16)
+    cbt = torch.randn(1, 1, t.G, 2, g, J, E, c, generator=gen).to(torch.bfloat16).float()
+    cbt[0, 0, 0, 1, :, :, 250] = cbt[0, 0, 0, 1, :, :, 3]        # codeword 250 == 3
+    m = 40
+    idx = torch.randint(0, E, (m, J), generator=gen)
+    idx[::3] = 250
+    xt = torch.empty(g, m, 1, t.head_dim)
+    for tau in range(g):
+        for jj in range(J):
+            xt[tau, :, 0, jj * c:(jj + 1) * c] = cbt[0, 0, 0, 1, tau, jj][idx[:, jj]]
+    pool = _run(t, 1, 0, 0, 1, xt.to(torch.bfloat16), None, cbt, np.arange(m, dtype=np.int64), 2)
+    got = _gpu_indices(pool, t, 0, 0, 1, np.arange(m))[:, 0].astype(np.int64)
+    expect = idx.numpy().copy()
+    expect[expect == 250] = 3
+    np.testing.assert_array_equal(got, expect)
