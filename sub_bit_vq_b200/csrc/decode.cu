@@ -60,7 +60,7 @@ constexpr int kRing = kPerHist >= 3 ? 2 : 4;   // index blocks in registers (rou
 constexpr int kPrefetchPages = 8;         // pages a warp asks L2 to fetch ahead of its loads
 constexpr float kRescaleSlack = 8.0f;     // log2 units a score may exceed m before m is raised
 constexpr int kFinishThreads = 256;
-constexpr int kWinChunk = 8;              // window tokens per warp per round of loads
+constexpr int kWinChunk = 9;              // window tokens per warp per round of loads (72 = 8 warps x 9)
 constexpr int kSpinLimit = 1 << 14;       // bounded mbarrier waits (each try sleeps up to kSuspendNs)
 constexpr uint32_t kSuspendNs = 65536u;
 
@@ -288,11 +288,14 @@ __device__ long long find_unit(const DecodeParams& p, long long u, int lane, int
 // Window partial of one pair over its n_win bf16 window tokens:
 // x_t = q . K_win[t] (log2 units), m = max x, l = sum 2^(x-m),
 // o = sum 2^(x-m) V_win[t]; written to res[0], res[1], res[2..2+D).
-// Every thread of the CTA (NWARPS warps) calls it; xwin holds n_win floats
-// and wpart NWARPS*D floats of shared memory. Ends with a barrier.
+// Every thread of the CTA (NWARPS warps) calls it. Warp w takes tokens
+// w, w + NWARPS, ..: it requests the key and value rows of up to kWinChunk
+// tokens at once, keeps its own running (m, l, o) and leaves it in
+// wstat[2w..2w+1] and wpart[w][D]; the warp partials are then merged.
+// Ends with a barrier.
 template <int D, int NWARPS>
 __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint16_t* qp,
-                               int n_win, float* xwin, float* wpart, float* res) {
+                               int n_win, float* wstat, float* wpart, float* res) {
   constexpr int NPL = (D / 2 + 31) / 32;               // bf16 channel pairs per lane
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (n_win <= 0) {                                    // CTA-uniform
@@ -312,17 +315,25 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
   const size_t head = (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * D;
   const unsigned int* wk = reinterpret_cast<const unsigned int*>(p.win_k + head);
   const unsigned int* wv = reinterpret_cast<const unsigned int*>(p.win_v + head);
+  float m = -INFINITY, l = 0.f;
+  float oacc[NPL][2];
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) oacc[k][0] = oacc[k][1] = 0.f;
   for (int t0 = warp; t0 < n_win; t0 += NWARPS * kWinChunk) {
-    uint32_t kr[kWinChunk][NPL];
+    uint32_t kr[kWinChunk][NPL], vr[kWinChunk][NPL];
 #pragma unroll
     for (int i = 0; i < kWinChunk; ++i) {
       const int t = t0 + i * NWARPS;
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
         const int pc = lane + 32 * k;
-        kr[i][k] = (t < n_win && pc < D / 2) ? __ldg(wk + static_cast<size_t>(t) * (D / 2) + pc) : 0u;
+        const bool ok = t < n_win && pc < D / 2;
+        kr[i][k] = ok ? __ldg(wk + static_cast<size_t>(t) * (D / 2) + pc) : 0u;
+        vr[i][k] = ok ? __ldg(wv + static_cast<size_t>(t) * (D / 2) + pc) : 0u;
       }
     }
+    float x[kWinChunk];
+    float mc = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kWinChunk; ++i) {
       float acc = 0.f;
@@ -331,36 +342,23 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
         const float2 kv = bf16x2_to_float2(kr[i][k]);
         acc = fmaf(qf[k][0], kv.x, fmaf(qf[k][1], kv.y, acc));
       }
-      acc = warp_sum(acc);
-      const int t = t0 + i * NWARPS;
-      if (lane == 0 && t < n_win) xwin[t] = acc;
+      x[i] = (t0 + i * NWARPS < n_win) ? warp_sum(acc) : -INFINITY;
+      mc = fmaxf(mc, x[i]);
     }
-  }
-  __syncthreads();
-  float m = -INFINITY;
-  for (int t = lane; t < n_win; t += 32) m = fmaxf(m, xwin[t]);
-  m = warp_max(m);
-  float l = 0.f;
-  for (int t = lane; t < n_win; t += 32) l += fast_exp2(xwin[t] - m);
-  l = warp_sum(l);
-  float oacc[NPL][2];
-#pragma unroll
-  for (int k = 0; k < NPL; ++k) oacc[k][0] = oacc[k][1] = 0.f;
-  for (int t0 = warp; t0 < n_win; t0 += NWARPS * kWinChunk) {
-    uint32_t vr[kWinChunk][NPL];
-#pragma unroll
-    for (int i = 0; i < kWinChunk; ++i) {
-      const int t = t0 + i * NWARPS;
+    if (mc > m) {                                      // warp-uniform
+      const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - mc);
+      l *= f;
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
-        const int pc = lane + 32 * k;
-        vr[i][k] = (t < n_win && pc < D / 2) ? __ldg(wv + static_cast<size_t>(t) * (D / 2) + pc) : 0u;
+        oacc[k][0] *= f;
+        oacc[k][1] *= f;
       }
+      m = mc;
     }
 #pragma unroll
     for (int i = 0; i < kWinChunk; ++i) {
-      const int t = t0 + i * NWARPS;
-      const float w = (t < n_win) ? fast_exp2(xwin[t] - m) : 0.f;
+      const float w = fast_exp2(x[i] - m);             // 0 past the window
+      l += w;
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
         const float2 vv = bf16x2_to_float2(vr[i][k]);
@@ -368,6 +366,10 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
         oacc[k][1] = fmaf(w, vv.y, oacc[k][1]);
       }
     }
+  }
+  if (lane == 0) {
+    wstat[2 * warp] = m;
+    wstat[2 * warp + 1] = l;
   }
 #pragma unroll
   for (int k = 0; k < NPL; ++k) {
@@ -378,15 +380,24 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
     }
   }
   __syncthreads();
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NWARPS; ++w) M = fmaxf(M, wstat[2 * w]);
+  float f[NWARPS];
+#pragma unroll
+  for (int w = 0; w < NWARPS; ++w) f[w] = (wstat[2 * w] == -INFINITY) ? 0.f : fast_exp2(wstat[2 * w] - M);
   for (int ch = tid; ch < D; ch += NWARPS * 32) {
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < NWARPS; ++w) o += wpart[w * D + ch];
+    for (int w = 0; w < NWARPS; ++w) o = fmaf(f[w], wpart[w * D + ch], o);
     res[2 + ch] = o;
   }
   if (tid == 0) {
-    res[0] = m;
-    res[1] = l;
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w) L = fmaf(f[w], wstat[2 * w + 1], L);
+    res[0] = M;
+    res[1] = L;
   }
   __syncthreads();
 }
@@ -438,6 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   const long long U = find_unit(p, -1, lane, &b_first, &pre_first);
   const long long u_lo = U * blockIdx.x / p.n_cta;
   const long long u_hi = U * (blockIdx.x + 1) / p.n_cta;
+  // the finish kernel may start its window work as SMs free up; it waits for
+  // this grid before it reads the records
+  asm volatile("griddepcontrol.launch_dependents;");
   if (u_lo >= u_hi) return;                            // CTA-uniform
   int b;
   long long pre;
@@ -730,7 +744,7 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
   constexpr int RS = 4 + kE * J;                       // record floats
   constexpr int JP = J + 1;                            // padded histogram row
   __shared__ float hs[kE * JP];
-  __shared__ float xwin[256];
+  __shared__ float wst[2 * NW];
   __shared__ float wpart[NW * D];
   __shared__ float wres[D + 2];
   __shared__ float ohist[D];
@@ -740,8 +754,14 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
   const int pair = blockIdx.x;
   const int b = pair / p.Hq, hq = pair % p.Hq, hkv = hq / p.ratio;
   const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
-  window_partial<D, NW>(p, b, hkv, p.q + static_cast<size_t>(pair) * D, min(N, p.W), xwin, wpart, wres);
   const int pages_b = seq_pages(p, b);                 // CTA-uniform
+  if (pages_b > 0 && tid < 32) {                       // the value slice, into L2 ahead of the contraction
+    const char* cv = reinterpret_cast<const char*>(p.cb_v + hkv * p.cb_stride_head);
+    constexpr uint32_t kSlice = kE * J * C * 4, kPiece = kSlice / 32;
+    static_assert(kSlice % (32 * 16) == 0, "prefetch pieces are 16-byte multiples");
+    prefetch_l2_bulk(cv + tid * kPiece, kPiece);
+  }
+  window_partial<D, NW>(p, b, hkv, p.q + static_cast<size_t>(pair) * D, min(N, p.W), wst, wpart, wres);
 
   // the pair's segment records: slots pair + c for the CTAs c that own its units
   int c_first = 0, c_last = -1;
@@ -761,6 +781,9 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
     c_first = static_cast<int>(((u0 + 1) * p.n_cta - 1) / U);
     c_last = static_cast<int>(((u0 + pages_b) * p.n_cta - 1) / U);
   }
+  // everything above reads only inputs; the segment records need the
+  // streaming kernel to be complete
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // a CTA whose unit range is empty wrote no record
   auto rec_of = [&](int c) -> const float* {
     return (U * c / p.n_cta < U * (c + 1) / p.n_cta)
@@ -899,7 +922,19 @@ loopvq_status launch_vq(const DecodeParams& p, cudaStream_t st, bool run_stream)
     vq_stream_kernel<J, C><<<p.n_cta, kThreads, kDynBytes, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return LOOPVQ_ERR_CUDA;
   }
-  vq_finish_kernel<J, C><<<p.B * p.Hq, kFinishThreads, 0, st>>>(p);
+  // programmatic dependent launch: the finish kernel's CTAs may start while
+  // the streaming kernel's last CTAs still run (griddepcontrol.wait inside)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.B * p.Hq));
+  cfg.blockDim = dim3(kFinishThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, vq_finish_kernel<J, C>, p) != cudaSuccess) return LOOPVQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
 }
 
