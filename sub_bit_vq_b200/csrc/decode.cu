@@ -505,11 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       const int n_rounds = (most_pages * bpp + 1) / 2;
       int i0 = 0;
       auto bt_entry = [&](int i) -> int { return (i < n_my_pages) ? bt[my_first + i * kNW] : -1; };
-      int bt_cur = bt_entry(lane);
+      int bt_cur = bt_entry(lane);                     // requested now, used after the slice lands
       int bt_nxt = bt_entry(32 + lane);
-      if (lane < kPrefetchPages && lane < n_my_pages && bt_cur >= 0 && bt_cur < p.n_pages)
-        prefetch_l2_bulk(pool_h + static_cast<int64_t>(bt_cur) * p.page_bytes,
-                         static_cast<uint32_t>(p.page_bytes));
       BlockRegs<J> ring[kRing] = {};
       // a cleared block keeps whatever bytes it held: every byte value
       // addresses a valid row, and base = -1 masks its scores and skips it
@@ -545,8 +542,6 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, p.Pg, blk,
                       lane, r);
       };
-#pragma unroll
-      for (int k = 0; k < kRing; ++k) issue(k, ring[k]);
 
       // ---- key LUT from the key slice staged in the histogram windows ----------
       if (tid < d) qs[tid] = qv;
@@ -559,8 +554,16 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         }
         cp_async_wait_all();
         __syncthreads();
+        if (j0 == 0) {                                 // the page table has landed: first index blocks
+          if (lane < kPrefetchPages && lane < n_my_pages && bt_cur >= 0 && bt_cur < p.n_pages)
+            prefetch_l2_bulk(pool_h + static_cast<int64_t>(bt_cur) * p.page_bytes,
+                             static_cast<uint32_t>(p.page_bytes));
+#pragma unroll
+          for (int k = 0; k < kRing; ++k) issue(k, ring[k]);
+        }
         // item = (tile of 32 rows, step): lane -> row tile*32 + lane, group
         // j0 + (step + lane) % JC, so the lanes' table stores hit distinct banks
+#pragma unroll 4
         for (int it = warp; it < (kE / 32) * JC; it += kNW) {
           const int e = (it / JC) * 32 + lane, jj = (it % JC + lane) % JC, j = j0 + jj;
           const float v = dot_c<C>(qs + j * C, stage + (static_cast<size_t>(jj) * kE + e) * C);
@@ -704,6 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         for (int h = 0; h < kNHist; ++h) fh[h] = (hm[h] == -INFINITY) ? 0.f : fast_exp2(hm[h] - Mh);
         // lane = column, rows warp + kNW*k; replicas of a group are summed
         const float* hist = stage;                     // the histogram windows as floats
+#pragma unroll 4
         for (int e = warp; e < kE; e += kNW) {
           float v = 0.f;
           if (lane_live) {
