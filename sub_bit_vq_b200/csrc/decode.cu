@@ -61,6 +61,7 @@ constexpr int kPrefetchPages = 8;         // pages a warp asks L2 to fetch ahead
 constexpr float kRescaleSlack = 8.0f;     // log2 units a score may exceed m before m is raised
 constexpr int kFinishThreads = 256;
 constexpr int kWinChunk = 9;              // window tokens per warp per round of loads (72 = 8 warps x 9)
+constexpr int kSegmentUnits = 16;        // work units (pages) charged for a segment's setup
 constexpr int kSpinLimit = 1 << 14;       // bounded mbarrier waits (each try sleeps up to kSuspendNs)
 constexpr uint32_t kSuspendNs = 65536u;
 
@@ -249,6 +250,11 @@ __device__ __forceinline__ int seq_pages(const DecodeParams& p, int b) {
   return min((n_vq + p.Pg - 1) / p.Pg, p.max_pages_per_seq);
 }
 
+// Work units of one (sequence, head) pair: its quantised pages, led by
+// kSegmentUnits units that stand for the setup of a segment. A CTA whose
+// range reaches into a second pair so takes fewer pages.
+__device__ __forceinline__ int pair_units(int pages) { return pages > 0 ? pages + kSegmentUnits : 0; }
+
 // Inclusive warp prefix sum.
 __device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
 #pragma unroll
@@ -260,8 +266,8 @@ __device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
 }
 
 // Walks sequences 0..B-1 (a warp at a time) to find the sequence whose
-// units [Hq*pre, Hq*(pre + pages)) contain unit `u` (or, with u < 0, just
-// the total). Returns the total number of units; *b_out, *pre_out describe
+// units [Hq*pre, Hq*(pre + pair_units)) contain unit `u` (or, with u < 0,
+// just the total). Returns the total number of units; *b_out, *pre_out describe
 // the hit (b_out = -1 if none).
 __device__ long long find_unit(const DecodeParams& p, long long u, int lane, int* b_out,
                                long long* pre_out) {
@@ -270,7 +276,7 @@ __device__ long long find_unit(const DecodeParams& p, long long u, int lane, int
   *pre_out = 0;
   for (int b0 = 0; b0 < p.B; b0 += 32) {
     const int b = b0 + lane;
-    const long long units = (b < p.B) ? static_cast<long long>(p.Hq) * seq_pages(p, b) : 0;
+    const long long units = (b < p.B) ? static_cast<long long>(p.Hq) * pair_units(seq_pages(p, b)) : 0;
     const long long incl = warp_incl_scan(units, lane);
     const long long excl = incl - units;
     const bool hit = units > 0 && acc + excl <= u && u < acc + incl;
@@ -456,10 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   int b;
   long long pre;
   find_unit(p, u_lo, lane, &b, &pre);
-  int pages_b = seq_pages(p, b);
+  int units_b = pair_units(seq_pages(p, b));
   const long long off = u_lo - static_cast<long long>(p.Hq) * pre;
-  int hq = static_cast<int>(off / pages_b);
-  int pg_start = static_cast<int>(off % pages_b);
+  int hq = static_cast<int>(off / units_b);
+  int pu_start = static_cast<int>(off % units_b);     // unit offset inside the pair
   long long u = u_lo;
 
   if (!bad_base) {
@@ -472,8 +478,10 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   bool wait_failed = false;
 
   while (u < u_hi && b < p.B) {
-    const int seg_pages = static_cast<int>(min(static_cast<long long>(pages_b - pg_start), u_hi - u));
-    const int pg_lo = pg_start, pg_hi = pg_start + seg_pages;
+    const int seg_units = static_cast<int>(min(static_cast<long long>(units_b - pu_start), u_hi - u));
+    // pages of this segment: its units past the pair's leading setup units
+    const int pg_lo = max(pu_start - kSegmentUnits, 0);
+    const int pg_hi = max(pu_start + seg_units - kSegmentUnits, 0);
     const int hkv = hq / p.ratio;
     const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
     const int n_vq = max(0, N - p.W);
@@ -482,6 +490,11 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       if (tid == 0) {
         rec[0] = NAN;
         rec[1] = 1.f;
+      }
+    } else if (pg_hi <= pg_lo) {                       // setup units only: an empty record
+      if (tid == 0) {
+        rec[0] = -INFINITY;
+        rec[1] = 0.f;
       }
     } else {
       const float* cbk = p.cb_k + hkv * p.cb_stride_head;
@@ -726,13 +739,13 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       }
     }
 
-    u += seg_pages;
-    pg_start = 0;
+    u += seg_units;
+    pu_start = 0;
     if (++hq == p.Hq) {
       hq = 0;
       do {
         ++b;
-      } while (b < p.B && u < u_hi && (pages_b = seq_pages(p, b)) == 0);
+      } while (b < p.B && u < u_hi && (units_b = pair_units(seq_pages(p, b))) == 0);
     }
   }
 }
@@ -774,16 +787,17 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
     int bb;
     long long pre;
     U = find_unit(p, -1, lane, &bb, &pre);
-    long long before = 0;                              // pages of sequences < b
+    long long before = 0;                              // units of one head of sequences < b
     for (int b0 = 0; b0 < b; b0 += 32) {
       const int bi = b0 + lane;
-      long long v = (bi < b) ? static_cast<long long>(seq_pages(p, bi)) : 0;
+      long long v = (bi < b) ? static_cast<long long>(pair_units(seq_pages(p, bi))) : 0;
       v = warp_incl_scan(v, lane);
       before += __shfl_sync(0xffffffffu, v, 31);
     }
-    const long long u0 = before * p.Hq + static_cast<long long>(hq) * pages_b;
+    const int units_b = pair_units(pages_b);
+    const long long u0 = before * p.Hq + static_cast<long long>(hq) * units_b;
     c_first = static_cast<int>(((u0 + 1) * p.n_cta - 1) / U);
-    c_last = static_cast<int>(((u0 + pages_b) * p.n_cta - 1) / U);
+    c_last = static_cast<int>(((u0 + units_b) * p.n_cta - 1) / U);
   }
   // everything above reads only inputs; the segment records need the
   // streaming kernel to be complete
