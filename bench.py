@@ -411,7 +411,7 @@ def encode_prefill(device, reps=3):
     return {"subvectors_per_s": nsub / sec, "ms_per_call": sec * 1e3,
             "shape": f"{n} tokens x {s.n_kv_heads} heads x {s.J} groups, D={s.D}, "
                      f"per-token LogNormal weights, one of K/V",
-            "kernel": "direct form (CUDA cores)"}
+            "kernel": "tcgen05 split-bf16 contraction + exact float32 rescore (tensor cores)"}
 
 
 # --------------------------------------------------------------------------

@@ -1,4 +1,7 @@
-// Nearest-centroid encoder, direct form (sm_100a CUDA cores).
+// Nearest-centroid encoder, direct form (sm_100a CUDA cores), and the
+// dispatch among the three encoder forms: a warp per token for the small
+// batches of the window eviction, this kernel for mid-sized batches, and the
+// tensor-core form (encode_tc.cu) for prefill-sized ones.
 //
 // One CTA = (tile of 128 tokens, channel group j, kv-head h). The CTA stages
 // the E x D codebook of (layer, h, gamma, K/V, j) in shared memory as
@@ -10,6 +13,7 @@
 // exact ties). The index byte goes to the rotated slot position of the pool.
 
 #include "common.cuh"
+#include "encode_common.cuh"
 #include "internal.h"
 
 namespace loopvq {
@@ -18,61 +22,7 @@ namespace {
 constexpr int kEncThreads = 128;
 constexpr int kEncWarpThreads = 256;    // small batches: one CTA per (group, head), a warp per token
 constexpr int kEncWarpMaxTokens = 64;   // batches up to this size take the warp form
-
-struct EncodeParams {
-  const uint16_t* x;            // bf16 bits
-  int64_t x_loop_stride, x_token_stride;
-  const float* w;               // nullable
-  int64_t w_loop_stride, w_token_stride;
-  const float* cb;              // codebooks at (layer, head 0, gamma, kv, tau 0)
-  int64_t cb_stride_head, cb_stride_loop;
-  const int64_t* slot_mapping;
-  uint8_t* pool;                // pool at (layer, head 0, gamma)
-  int64_t pool_stride_head, page_bytes, plane_bytes;
-  int64_t n_slots;              // n_pages * Pg
-  int n_tokens, d, Pg, J, LB, GR, kv;
-};
-
-// Writes index `e` of (slot, group j, head h) to its byte in the pool.
-__device__ __forceinline__ void store_index(const EncodeParams& p, int64_t slot, int j, int h, int e) {
-  const int64_t page = slot / p.Pg;
-  const int sl = static_cast<int>(slot % p.Pg);
-  int64_t off;
-  if (p.kv == 0) {                          // K plane: rotated slot rows
-    const int blk = sl / p.LB, rot = sl % p.LB;
-    int pos = j - rot % p.J;
-    if (pos < 0) pos += p.J;
-    off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR + rot * p.GR +
-          pos % p.GR;
-  } else {                                  // V plane: group-major
-    off = static_cast<int64_t>(j) * p.Pg + sl;
-  }
-  p.pool[h * p.pool_stride_head + page * p.page_bytes + p.kv * p.plane_bytes + off] =
-      static_cast<uint8_t>(e);
-}
-
-// Loads token n's sub-vector of (group j, head h) and its weights (1 when
-// no weights are given).
-template <int C, int G>
-__device__ __forceinline__ void load_subvector(const EncodeParams& p, int n, int j, int h,
-                                               float (&s)[C * G], float (&w)[C * G]) {
-#pragma unroll
-  for (int tau = 0; tau < G; ++tau) {
-    const uint16_t* xr = p.x + tau * p.x_loop_stride + n * p.x_token_stride +
-                         static_cast<int64_t>(h) * p.d + j * C;
-#pragma unroll
-    for (int ch = 0; ch < C; ++ch) s[tau * C + ch] = bf16_bits_to_float(xr[ch]);
-    if (p.w != nullptr) {
-      const float* wr = p.w + tau * p.w_loop_stride + n * p.w_token_stride +
-                        static_cast<int64_t>(h) * p.d + j * C;
-#pragma unroll
-      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = wr[ch];
-    } else {
-#pragma unroll
-      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = 1.f;
-    }
-  }
-}
+constexpr int kEncTcMinTokens = 2048;   // batches from this size take the tensor-core form
 
 // Small batches (the tokens leaving the recent window at each decode step):
 // one CTA per (group j, head h) stages the codebook of (j, h) once as
@@ -177,6 +127,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
 
 template <int C, int G>
 loopvq_status launch_enc(const EncodeParams& p, int J, int H, cudaStream_t st) {
+  if (p.n_tokens >= kEncTcMinTokens && encode_tc_supported(C, G))
+    return launch_encode_tc(p, C, G, J, H, st);
   if (p.n_tokens <= kEncWarpMaxTokens) {
     encode_warp_kernel<C, G><<<dim3(J, H), kEncWarpThreads, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;

@@ -1,0 +1,70 @@
+// Pieces shared by the encoder kernels (direct form and tensor-core form).
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+#include "loopvq.h"
+
+namespace loopvq {
+
+struct EncodeParams {
+  const uint16_t* x;            // bf16 bits
+  int64_t x_loop_stride, x_token_stride;
+  const float* w;               // nullable
+  int64_t w_loop_stride, w_token_stride;
+  const float* cb;              // codebooks at (layer, head 0, gamma, kv, tau 0)
+  int64_t cb_stride_head, cb_stride_loop;
+  const int64_t* slot_mapping;
+  uint8_t* pool;                // pool at (layer, head 0, gamma)
+  int64_t pool_stride_head, page_bytes, plane_bytes;
+  int64_t n_slots;              // n_pages * Pg
+  int n_tokens, d, Pg, J, LB, GR, kv;
+};
+
+// Writes index `e` of (slot, group j, head h) to its byte in the pool.
+__device__ __forceinline__ void store_index(const EncodeParams& p, int64_t slot, int j, int h, int e) {
+  const int64_t page = slot / p.Pg;
+  const int sl = static_cast<int>(slot % p.Pg);
+  int64_t off;
+  if (p.kv == 0) {                          // K plane: rotated slot rows
+    const int blk = sl / p.LB, rot = sl % p.LB;
+    int pos = j - rot % p.J;
+    if (pos < 0) pos += p.J;
+    off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR + rot * p.GR +
+          pos % p.GR;
+  } else {                                  // V plane: group-major
+    off = static_cast<int64_t>(j) * p.Pg + sl;
+  }
+  p.pool[h * p.pool_stride_head + page * p.page_bytes + p.kv * p.plane_bytes + off] =
+      static_cast<uint8_t>(e);
+}
+
+// Loads token n's sub-vector of (group j, head h) and its weights (1 when
+// no weights are given).
+template <int C, int G>
+__device__ __forceinline__ void load_subvector(const EncodeParams& p, int n, int j, int h,
+                                               float (&s)[C * G], float (&w)[C * G]) {
+#pragma unroll
+  for (int tau = 0; tau < G; ++tau) {
+    const uint16_t* xr = p.x + tau * p.x_loop_stride + n * p.x_token_stride +
+                         static_cast<int64_t>(h) * p.d + j * C;
+#pragma unroll
+    for (int ch = 0; ch < C; ++ch) s[tau * C + ch] = bf16_bits_to_float(xr[ch]);
+    if (p.w != nullptr) {
+      const float* wr = p.w + tau * p.w_loop_stride + n * p.w_token_stride +
+                        static_cast<int64_t>(h) * p.d + j * C;
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = wr[ch];
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = 1.f;
+    }
+  }
+}
+
+// Launches the tensor-core encoder (D = c*g in {8, 16, 32}); see encode_tc.cu.
+bool encode_tc_supported(int c, int g);
+loopvq_status launch_encode_tc(const EncodeParams& p, int c, int g, int J, int H, void* stream);
+
+}  // namespace loopvq

@@ -209,3 +209,48 @@ def test_small_batch_j12_and_ties():
     expect = idx.numpy().copy()
     expect[expect == 250] = 3
     np.testing.assert_array_equal(got, expect)
+
+
+@pytest.mark.parametrize("per_token", [True, False])
+def test_prefill_batches_take_the_tensor_core_form(per_token):
+    # batches of 2048 tokens and more: tcgen05 contraction plus exact rescore
+    s = W128
+    n, n_pages, layer, gamma, kv = 2100, 40, 0, 1, 0
+    x = loop_group_kv(s, layer, gamma, kv, n)
+    w = weights(s, n, per_token, layer, gamma, kv)
+    cb = random_codebooks(s, 2, 21)
+    slots = _slots(n, n_pages, s.page_tokens, 22, skip_every=11)
+    pool = _run(s, 2, layer, gamma, kv, x, w, cb, slots, n_pages)
+    _, dist = O.encode_group_ref(x.double().numpy(), cb[layer, :, gamma, kv].double().numpy(),
+                                 w.double().numpy())
+    keep = slots >= 0
+    check_indices(_gpu_indices(pool, s, layer, gamma, kv, slots)[keep], dist[keep])
+
+
+def test_prefill_tensor_core_j12_fitted_and_ties():
+    s = J12
+    n, n_pages = 2304, 26
+    x = loop_group_kv(s, 0, 0, 1, n)
+    cb = codebooks_for_layer(s, 0, n_samples=2048, iters=8)[None]
+    slots = _slots(n, n_pages, s.page_tokens, 23)
+    pool = _run(s, 1, 0, 0, 1, x, None, cb, slots, n_pages)
+    _, dist = O.encode_group_ref(x.double().numpy(), cb[0, :, 0, 1].double().numpy())
+    check_indices(_gpu_indices(pool, s, 0, 0, 1, slots), dist)
+    # exact codewords with a duplicated codeword through the tensor-core form
+    t = W128.with_(n_kv_heads=1, n_q_heads=1)
+    g, J, c, E = t.loop_group, t.J, t.chan_group, 256
+    gen = torch.Generator().manual_seed(24)
+    cbt = torch.randn(1, 1, t.G, 2, g, J, E, c, generator=gen).to(torch.bfloat16).float()
+    cbt[0, 0, 0, 0, :, :, 99] = cbt[0, 0, 0, 0, :, :, 5]          # codeword 99 == 5
+    m = 2048
+    idx = torch.randint(0, E, (m, J), generator=gen)
+    idx[::7] = 99
+    xt = torch.empty(g, m, 1, t.head_dim)
+    for tau in range(g):
+        for jj in range(J):
+            xt[tau, :, 0, jj * c:(jj + 1) * c] = cbt[0, 0, 0, 0, tau, jj][idx[:, jj]]
+    pool = _run(t, 1, 0, 0, 0, xt.to(torch.bfloat16), None, cbt, np.arange(m, dtype=np.int64), 33)
+    got = _gpu_indices(pool, t, 0, 0, 0, np.arange(m))[:, 0].astype(np.int64)
+    expect = idx.numpy().copy()
+    expect[expect == 99] = 5
+    np.testing.assert_array_equal(got, expect)
