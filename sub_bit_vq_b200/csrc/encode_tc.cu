@@ -14,8 +14,10 @@
 // tcgen05.mma chain that leaves S (128 x 256, fp32) in tensor memory, and
 // each thread reads its row back with tcgen05.ld. Operands are bf16 split
 // into high and low parts, a.b ~= a_hi.b_hi + a_hi.b_lo + a_lo.b_hi (K' =
-// 6D), whose error stays far below
-//     margin = 2^-11 * (sum_i |a_i| max_e |b_ei| + sum_i w_i s_i^2).
+// 6D): each S_e is off by at most about 2^-14.3 * sum_i |a_i b_ei| (the
+// dropped lo*lo terms, the split residuals, fp32 accumulation over K'), so
+// twice that, plus the direct form's own rounding, stays below
+//     margin = 2^-12 * (sum_i |a_i| max_e |b_ei| + sum_i w_i s_i^2).
 // Every centroid whose S_e is within the margin of the row's minimum is
 // rescored with the float32 direct form and term order of encode_kernel;
 // the first minimum of those (smallest index on equal distances) is the
@@ -178,17 +180,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
   const uint32_t my_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const int n_tiles = (p.n_tokens + kTcRows - 1) / kTcRows;
   bool failed = false;
+  // this thread's token of the next tile, requested one tile ahead
+  float s_nx[D], w_nx[D];
+  int64_t slot_nx = -1;
+  auto fetch = [&](int t) {
+    const int n = t * kTcRows + tid;
+    slot_nx = (t < n_tiles && n < p.n_tokens) ? p.slot_mapping[n] : -1;
+    if (slot_nx >= 0 && slot_nx < p.n_slots) load_subvector<C, G>(p, n, j, h, s_nx, w_nx);
+  };
+  fetch(0);
   for (int t = 0; t < n_tiles; ++t) {
     // ---- this thread's row of A ----------------------------------------------
-    const int n = t * kTcRows + tid;
-    int64_t slot = -1;
+    const int64_t slot = slot_nx;
     float s[D], w[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      s[i] = s_nx[i];
+      w[i] = w_nx[i];
+    }
     float a[K2];
     float margin = 0.f;
-    if (n < p.n_tokens) slot = p.slot_mapping[n];
     const bool live = slot >= 0 && slot < p.n_slots;
     if (live) {
-      load_subvector<C, G>(p, n, j, h, s, w);
       float ms = 0.f, wss = 0.f;
 #pragma unroll
       for (int i = 0; i < D; ++i) {
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
       }
 #pragma unroll
       for (int i = 0; i < K2; ++i) ms = fmaf(fabsf(a[i]), bm[i], ms);
-      margin = ldexpf(ms + wss, -11);
+      margin = ldexpf(ms + wss, -12);
     } else {
 #pragma unroll
       for (int i = 0; i < K2; ++i) a[i] = 0.f;
@@ -222,6 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                    ::"r"(mbar_a) : "memory");
     }
+    fetch(t + 1);                                    // lands while the tensor cores work
     bool done = failed;
     for (int it = 0; it < kTcSpin && !done; ++it) {
       uint32_t ok;
