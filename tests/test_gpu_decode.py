@@ -104,3 +104,33 @@ def test_full_long_context_config_sampled():
     check_decode(case, out, lse, torch.bfloat16, pairs=pairs)
     out, lse = case.run_gpu(torch.float32)
     check_decode(case, out, lse, torch.float32, pairs=pairs)
+
+
+# Every (J, c) instantiation the library dispatches, beyond the shapes above:
+# J = 8 (four replicas per group in a 32-slot block), J = 24 (24-slot blocks,
+# lanes 24..31 idle) and the c = 2 forms.
+OTHER_SHAPES = [
+    Shape("j8c4", n_layers=1, n_kv_heads=2, n_q_heads=2, head_dim=32, n_loops=4, loop_group=4,
+          chan_group=4, batch=3, context=0, seed=31),
+    Shape("j8c8", n_layers=1, n_kv_heads=1, n_q_heads=2, head_dim=64, n_loops=4, loop_group=4,
+          chan_group=8, batch=3, context=0, seed=32),
+    Shape("j24c4", n_layers=1, n_kv_heads=2, n_q_heads=2, head_dim=96, n_loops=4, loop_group=4,
+          chan_group=4, batch=3, context=0, page_tokens=96, seed=33),
+    Shape("j16c8", n_layers=1, n_kv_heads=1, n_q_heads=2, head_dim=128, n_loops=4, loop_group=4,
+          chan_group=8, batch=3, context=0, seed=38),
+    Shape("j32c2", n_layers=1, n_kv_heads=2, n_q_heads=2, head_dim=64, n_loops=4, loop_group=4,
+          chan_group=2, batch=3, context=0, seed=34),
+    Shape("j24c2", n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=48, n_loops=4, loop_group=4,
+          chan_group=2, batch=3, context=0, page_tokens=96, seed=35),
+    Shape("j12c2", n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=24, n_loops=4, loop_group=4,
+          chan_group=2, batch=3, context=0, page_tokens=48, seed=36),
+    Shape("j16c2", n_layers=1, n_kv_heads=2, n_q_heads=2, head_dim=32, n_loops=4, loop_group=4,
+          chan_group=2, batch=3, context=0, seed=37),
+]
+
+
+@pytest.mark.parametrize("shape", OTHER_SHAPES, ids=lambda s: s.name)
+def test_every_dispatched_group_shape(shape):
+    case = DecodeCase(shape, [73, 640, 2500], loop_step=2, seed=40)
+    out, lse = case.run_gpu(torch.float32)
+    check_decode(case, out, lse, torch.float32)

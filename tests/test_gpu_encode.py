@@ -254,3 +254,18 @@ def test_prefill_tensor_core_j12_fitted_and_ties():
     expect = idx.numpy().copy()
     expect[expect == 99] = 5
     np.testing.assert_array_equal(got, expect)
+
+
+def test_prefill_tensor_core_d8():
+    # c = 2, g = 4: 8-element sub-vectors, K' = 48
+    s = Shape("c2enc", n_layers=1, n_kv_heads=2, n_q_heads=2, head_dim=64, n_loops=4, loop_group=4,
+              chan_group=2, batch=1, context=0, seed=203)
+    n, n_pages = 2200, 36
+    x = loop_group_kv(s, 0, 0, 0, n)
+    w = weights(s, n, True, 0, 0, 0)
+    cb = random_codebooks(s, 1, 25)
+    slots = _slots(n, n_pages, s.page_tokens, 26)
+    pool = _run(s, 1, 0, 0, 0, x, w, cb, slots, n_pages)
+    _, dist = O.encode_group_ref(x.double().numpy(), cb[0, :, 0, 0].double().numpy(),
+                                 w.double().numpy())
+    check_indices(_gpu_indices(pool, s, 0, 0, 0, slots), dist)
