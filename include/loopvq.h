@@ -185,8 +185,8 @@ loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_
 /*
  * Bytes of scratch that loopvq_decode_attn needs for `batch` sequences of
  * at most `max_seq_len` tokens: (batch*Hq + 256) segment records of
- * 4 + 256*J float32 (a segment's softmax maximum and sum and its value
- * histogram). Host only, pure.
+ * 4 + head_dim float32 (a segment's softmax maximum and sum and its
+ * unnormalised output). Host only, pure.
  */
 size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int max_seq_len);
 
@@ -250,7 +250,7 @@ loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_s
  * kernels overlap on the GPU, e.g. on two streams without ordering, race
  * on it and give undefined results.
  */
-#define LOOPVQ_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+#define LOOPVQ_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
 loopvq_status loopvq_decode_attn_noalloc(const loopvq_config* cfg, int layer, int loop_step,
                                          int batch, int max_seq_len, const void* q,
                                          const uint8_t* pool, const float* codebooks,

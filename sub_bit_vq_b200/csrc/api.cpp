@@ -167,11 +167,11 @@ loopvq_status loopvq_cache_layout(const loopvq_config* cfg, loopvq_layout* out) 
 size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int max_seq_len) {
   Geometry g;
   if (loopvq::make_geometry(cfg, &g) != LOOPVQ_OK || batch <= 0 || max_seq_len < 0) return 0;
-  // one record (m, l, two spare floats, value histogram W[E][J]) per
+  // one record (m, l, two spare floats, unnormalised output o[d]) per
   // (pair, streaming CTA) segment: record slots pair + cta never collide, so
   // pairs + CTAs slots suffice
   const size_t slots = static_cast<size_t>(batch) * g.Hq + loopvq::kMaxStreamCtas;
-  return slots * (4 + static_cast<size_t>(g.E) * g.J) * sizeof(float);
+  return slots * (4 + static_cast<size_t>(g.d)) * sizeof(float);
 }
 
 loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_idx, int kv,

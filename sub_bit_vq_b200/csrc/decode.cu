@@ -25,13 +25,14 @@
 //      and weights before its turn and only the histogram updates inside it.
 //      Each histogram keeps one running maximum m, raised only when a vote
 //      finds a score above m + kRescaleSlack.
-//   3. The four histograms are merged into the segment record
-//      (m, l, W[E][J]) at slot (pair + cta).
+//   3. The four histograms are merged with log-sum-exp weights into W[E][J],
+//      which is contracted with the value codebook slice,
+//      o_j = sum_e W[e][j] C_V[j][e][tau]; the segment record (m, l, o[d]) goes
+//      to slot (pair + cta).
 //
 // vq_finish_kernel: one CTA per pair scores the bf16 window tokens (prefix +
-// recent), merges the pair's segment histograms with log-sum-exp weights,
-// contracts the merged histogram with the value codebook slice,
-// o_j = sum_e W[e][j] C_V[j][e][tau], and writes out and lse.
+// recent), merges them with the pair's segment records (log-sum-exp
+// weights) and writes out and lse.
 //
 // The hot loops address shared memory by absolute shared-window address, so
 // that one byte permute of an index word gives a complete address: the
@@ -89,7 +90,7 @@ struct DecodeParams {
   const int32_t* seq_lens;
   const uint16_t* win_k;            // bf16 bits [B][Hkv][W][d]
   const uint16_t* win_v;
-  float* records;                   // [pairs + n_cta][4 + E*J]: m, l, -, -, W[E][J]
+  float* records;                   // [pairs + n_cta][4 + d]: m, l, -, -, o[d]
   void* out;
   float* lse;
   int B, Hq, Hkv, ratio, W, Pg, n_pages, max_pages_per_seq, max_seq_len;
@@ -413,7 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   using T = Traits<J>;
   constexpr int d = J * C;
   constexpr int LB = T::LB;
-  constexpr int RS = 4 + kE * J;                       // record floats
+  constexpr int RS = 4 + d;                            // record floats
+  constexpr int EP = kE + 1;                           // padded row of the transposed merged histogram
+  static_assert(J * EP * 4 <= static_cast<int>(kHistEnd - kHistAbs), "merged histogram fits the windows");
   // groups of the key slice staged at once in the (empty) histogram windows
   constexpr int JC = (J * kE * C * 4 <= static_cast<int>(kHistEnd - kHistAbs))
                          ? J : static_cast<int>(kHistEnd - kHistAbs) / (kE * C * 4);
@@ -502,6 +505,12 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       __syncthreads();                                 // previous segment done with LUT and histograms
       // the first chunk of the key slice goes out before anything that waits
       for (int i = tid * 4; i < JC * kE * C; i += kThreads * 4) cp_async16(stage + i, cbk + i);
+      const float* cbv = p.cb_v + hkv * p.cb_stride_head;
+      if (warp == kNW - 1) {                           // the value slice, into L2 for the contraction
+        constexpr uint32_t kSlice = kE * J * C * 4, kPiece = kSlice / 32;
+        static_assert(kSlice % (32 * 16) == 0, "prefetch pieces are 16-byte multiples");
+        prefetch_l2_bulk(reinterpret_cast<const char*>(cbv) + lane * kPiece, kPiece);
+      }
       const float qv = (tid < d) ? bf16_bits_to_float(qp[tid]) * p.scale_log2 : 0.f;
 
       // ---- index ring prologue ----------------------------------------------
@@ -607,13 +616,12 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           if (!lane_live) return;
         }
         pp += (lane / J) * J;
+        float4 p4 = *reinterpret_cast<const float4*>(pp);
 #pragma unroll
         for (int i = 0; i < J; i += 4) {
           const uint32_t w = r.v[i >> 2];
           const uint32_t a0 = __byte_perm(w, hx, 0x7604u), a1 = __byte_perm(w, hx, 0x7614u);
           const uint32_t a2 = __byte_perm(w, hx, 0x7624u), a3 = __byte_perm(w, hx, 0x7634u);
-          const float o0 = lds_h(a0), o1 = lds_h(a1), o2 = lds_h(a2), o3 = lds_h(a3);
-          const float4 p4 = *reinterpret_cast<const float4*>(pp + i);
           // fold each weight into the last slot of the four with the same row
           float q1 = p4.y, q2 = p4.z, q3 = p4.w;
           if (a1 == a0) q1 += p4.x;
@@ -622,10 +630,14 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           if (a3 == a0) q3 += p4.x;
           if (a3 == a1) q3 += p4.y;
           if (a3 == a2) q3 += p4.z;
+          const float o0 = lds_h(a0), o1 = lds_h(a1), o2 = lds_h(a2), o3 = lds_h(a3);
+          // the next batch's weights (never written during the pass) before this batch's stores
+          const float4 p4n = (i + 4 < J) ? *reinterpret_cast<const float4*>(pp + i + 4) : p4;
           sts_h(a0, o0 + p4.x);
           sts_h(a1, o1 + q1);
           sts_h(a2, o2 + q2);
           sts_h(a3, o3 + q3);
+          p4 = p4n;
         }
       };
       // One round: key scores and (against the maximum this warp saw last)
@@ -701,13 +713,13 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       }
       __syncthreads();
 
-      // ---- merge the histograms into the segment record ---------------------------
+      // ---- merge the histograms, contract with the value slice -------------------
       float Mh = -INFINITY;
 #pragma unroll
       for (int h = 0; h < kNHist; ++h) Mh = fmaxf(Mh, hm[h]);
       if (Mh == -INFINITY) {                           // nothing valid: an empty record
         if (tid == 0) {
-          rec[0] = -INFINITY;
+          rec[0] = (flags[0] != 0) ? NAN : -INFINITY;
           rec[1] = 0.f;
         }
       } else {
@@ -718,19 +730,56 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         float fh[kNHist];
 #pragma unroll
         for (int h = 0; h < kNHist; ++h) fh[h] = (hm[h] == -INFINITY) ? 0.f : fast_exp2(hm[h] - Mh);
-        // lane = column, rows warp + kNW*k; replicas of a group are summed
+        // W[e][j]: lane = column, rows warp + kNW*k; replicas of a group are summed
+        constexpr int NR = (kE + kNW - 1) / kNW;       // rows per warp
         const float* hist = stage;                     // the histogram windows as floats
-#pragma unroll 4
-        for (int e = warp; e < kE; e += kNW) {
+        float wv[NR];
+#pragma unroll
+        for (int k = 0; k < NR; ++k) {
+          const int e = warp + kNW * k;
           float v = 0.f;
-          if (lane_live) {
+          if (e < kE && lane_live) {
 #pragma unroll
             for (int h = 0; h < kNHist; ++h)
               v = fmaf(fh[h], hist[(h >> 1) * 16384 + e * 64 + (h & 1) * 32 + lane], v);
           }
 #pragma unroll
           for (int o = (T::R / 2) * J; o >= J; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-          if (lane < J) rec[4 + e * J + lane] = v;
+          wv[k] = v;
+        }
+        __syncthreads();                               // every histogram word read
+        // transposed, padded: wt[j*EP + e] (lanes of a row and of a column hit distinct banks)
+        float* wt = stage;
+#pragma unroll
+        for (int k = 0; k < NR; ++k) {
+          const int e = warp + kNW * k;
+          if (e < kE && lane < J) wt[lane * EP + e] = wv[k];
+        }
+        __syncthreads();
+        // o[j*C + ch] = sum_e W[e][j] C_V[j][e][ch]: warp -> groups, lane -> rows lane + 32 i
+        constexpr int JPW = (J + kNW - 1) / kNW;
+#pragma unroll 1
+        for (int jw = 0; jw < JPW; ++jw) {
+          const int j = warp + kNW * jw;
+          if (j >= J) break;                           // warp-uniform
+          float cv[kE / 32][C];
+#pragma unroll
+          for (int i = 0; i < kE / 32; ++i)
+            load_cw<C>(cbv + (static_cast<size_t>(j) * kE + lane + 32 * i) * C, cv[i]);
+          float acc[C];
+#pragma unroll
+          for (int ch = 0; ch < C; ++ch) acc[ch] = 0.f;
+#pragma unroll
+          for (int i = 0; i < kE / 32; ++i) {
+            const float h = wt[j * EP + lane + 32 * i];
+#pragma unroll
+            for (int ch = 0; ch < C; ++ch) acc[ch] = fmaf(h, cv[i][ch], acc[ch]);
+          }
+#pragma unroll
+          for (int ch = 0; ch < C; ++ch) {
+            const float t = warp_sum(acc[ch]);
+            if (lane == ch) rec[4 + j * C + ch] = t;
+          }
         }
         if (tid == 0) {
           rec[0] = (flags[0] != 0) ? NAN : Mh;         // a turn that timed out poisons the pair
@@ -750,21 +799,16 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   }
 }
 
-// One CTA per (sequence, query head): the bf16 window partial, the merge of
-// the pair's segment histograms (log-sum-exp weights) and their contraction
-// with the value codebook slice, o_j = sum_e W[e][j] C_V[j][e][tau]; writes
-// out and lse.
+// One CTA per (sequence, query head): the bf16 window partial and the merge
+// of the pair's segment records (log-sum-exp weights); writes out and lse.
 template <int J, int C>
 __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeParams p) {
   constexpr int D = J * C;
   constexpr int NW = kFinishThreads / 32;
-  constexpr int RS = 4 + kE * J;                       // record floats
-  constexpr int JP = J + 1;                            // padded histogram row
-  __shared__ float hs[kE * JP];
+  constexpr int RS = 4 + D;                            // record floats
   __shared__ float wst[2 * NW];
   __shared__ float wpart[NW * D];
   __shared__ float wres[D + 2];
-  __shared__ float ohist[D];
   __shared__ float fc[kMaxStreamCtas];
   __shared__ float sstat[4];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -772,12 +816,6 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
   const int b = pair / p.Hq, hq = pair % p.Hq, hkv = hq / p.ratio;
   const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
   const int pages_b = seq_pages(p, b);                 // CTA-uniform
-  if (pages_b > 0 && tid < 32) {                       // the value slice, into L2 ahead of the contraction
-    const char* cv = reinterpret_cast<const char*>(p.cb_v + hkv * p.cb_stride_head);
-    constexpr uint32_t kSlice = kE * J * C * 4, kPiece = kSlice / 32;
-    static_assert(kSlice % (32 * 16) == 0, "prefetch pieces are 16-byte multiples");
-    prefetch_l2_bulk(cv + tid * kPiece, kPiece);
-  }
   window_partial<D, NW>(p, b, hkv, p.q + static_cast<size_t>(pair) * D, min(N, p.W), wst, wpart, wres);
 
   // the pair's segment records: slots pair + c for the CTAs c that own its units
@@ -811,16 +849,19 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
     float M = wres[0];
     for (int c = c_first + lane; c <= c_last; c += 32) {
       const float* rec = rec_of(c);
-      if (rec != nullptr) M = fmaxf(M, rec[0]);
+      if (rec != nullptr) M = fmaxf(M, __ldcg(rec));
     }
     M = warp_max(M);
     float L = 0.f;
     for (int c = c_first + lane; c <= c_last; c += 32) {
       const float* rec = rec_of(c);
       float f = 0.f;
-      if (rec != nullptr && rec[0] != -INFINITY) {
-        f = fast_exp2(rec[0] - M);
-        L += rec[1] * f;
+      if (rec != nullptr) {
+        const float m = __ldcg(rec);
+        if (m != -INFINITY) {
+          f = fast_exp2(m - M);                          // NaN m (a timed-out turn) poisons M and L
+          L += __ldcg(rec + 1) * f;
+        }
       }
       fc[c - c_first] = f;
     }
@@ -834,78 +875,13 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
   }
   __syncthreads();
   const float M = sstat[0], L = sstat[1], f_win = sstat[2];
-  bool any_hist = false;
-  for (int c = c_first; c <= c_last; ++c) any_hist |= fc[c - c_first] != 0.f;
-  if (any_hist) {                                      // CTA-uniform
-    // every thread owns the same PER words of each record: a record's words
-    // are requested together, one record after another
-    constexpr int PER = (kE * J + kFinishThreads - 1) / kFinishThreads;
-    float hacc[PER];
-#pragma unroll
-    for (int k = 0; k < PER; ++k) hacc[k] = 0.f;
-    for (int c = c_first; c <= c_last; ++c) {
-      const float f = fc[c - c_first];
-      if (f == 0.f) continue;                          // CTA-uniform
-      const float* r = p.records + static_cast<size_t>(pair + c) * RS + 4;
-      float v[PER];
-#pragma unroll
-      for (int k = 0; k < PER; ++k) {
-        const int i = tid + k * kFinishThreads;
-        v[k] = (i < kE * J) ? __ldcg(r + i) : 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < PER; ++k) hacc[k] = fmaf(f, v[k], hacc[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < PER; ++k) {
-      const int i = tid + k * kFinishThreads;
-      if (i < kE * J) hs[(i / J) * JP + i % J] = hacc[k];
-    }
-    __syncthreads();
-    // warp -> groups j = warp, warp + NW, ..; lane -> rows lane + 32*i
-    const float* cbv = p.cb_v + hkv * p.cb_stride_head;
-    constexpr int JPW = (J + NW - 1) / NW;             // groups per warp
-    constexpr int JCH = (C >= 8 && JPW > 2) ? 2 : JPW; // groups whose codewords load together
-#pragma unroll 1
-    for (int j0 = 0; j0 < JPW; j0 += JCH) {
-      float cv[JCH][kE / 32][C];
-#pragma unroll
-      for (int jj = 0; jj < JCH; ++jj) {
-        const int j = warp + NW * (j0 + jj);
-        if (j < J) {
-#pragma unroll
-          for (int i = 0; i < kE / 32; ++i)
-            load_cw<C>(cbv + (static_cast<size_t>(j) * kE + lane + 32 * i) * C, cv[jj][i]);
-        }
-      }
-#pragma unroll
-      for (int jj = 0; jj < JCH; ++jj) {
-        const int j = warp + NW * (j0 + jj);
-        if (j >= J) continue;                          // warp-uniform
-        float acc[C];
-#pragma unroll
-        for (int ch = 0; ch < C; ++ch) acc[ch] = 0.f;
-#pragma unroll
-        for (int i = 0; i < kE / 32; ++i) {
-          const float h = hs[(lane + 32 * i) * JP + j];
-#pragma unroll
-          for (int ch = 0; ch < C; ++ch) acc[ch] = fmaf(h, cv[jj][i][ch], acc[ch]);
-        }
-#pragma unroll
-        for (int ch = 0; ch < C; ++ch) {
-          const float t = warp_sum(acc[ch]);
-          if (lane == 0) ohist[j * C + ch] = t;
-        }
-      }
-    }
-  } else {
-    for (int i = tid; i < D; i += kFinishThreads) ohist[i] = 0.f;
-  }
-  __syncthreads();
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
   for (int ch = tid; ch < D; ch += kFinishThreads) {
-    float o = ohist[ch];
-    if (f_win != 0.f) o = fmaf(f_win, wres[2 + ch], o);
+    float o = (f_win != 0.f) ? f_win * wres[2 + ch] : 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+      const float f = fc[c - c_first];
+      if (f != 0.f) o = fmaf(f, __ldcg(p.records + static_cast<size_t>(pair + c) * RS + 4 + ch), o);
+    }
     o *= inv;
     if (p.out_dtype == LOOPVQ_DTYPE_F32)
       static_cast<float*>(p.out)[static_cast<size_t>(pair) * D + ch] = o;

@@ -144,7 +144,7 @@ def test_workspace_bytes_formula():
     # one record (m, l, 2 spare, value histogram [256][J]) of float32 per
     # (sequence, query head, split)
     n = L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64)
-    rec = 4 * (4 + 256 * (cfg.head_dim // cfg.chan_group))
+    rec = 4 * (4 + cfg.head_dim)
     assert n % rec == 0 and n >= rec * 2 * cfg.n_q_heads
     # more sequences need more records
     assert L.loopvq_decode_workspace_bytes(cfg, 4, 72 + 5 * 64) > n
