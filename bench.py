@@ -414,6 +414,60 @@ def encode_prefill(device, reps=3):
             "kernel": "tcgen05 split-bf16 contraction + exact float32 rescore (tensor cores)"}
 
 
+def kmeans_step(device, reps=3):
+    """One weighted Lloyd step of the codebooks of one (layer, loop group,
+    K/V) on the 32768-token prefill sample: the assignment (the encoder,
+    writing indices to an array) plus the weighted centroid update. The
+    update kernel is timed alone too, against the HBM bytes it must move."""
+    import torch
+
+    import sub_bit_vq_b200 as L
+    from synthetic import SHAPES, codebooks_for_layer, loop_group_kv, weights
+
+    s = SHAPES["sweep"]
+    n = 32768
+    cfg = L.LoopVQConfig(n_layers=1, n_kv_heads=s.n_kv_heads, n_q_heads=s.n_q_heads,
+                         head_dim=s.head_dim, n_loops=s.n_loops, loop_group=s.loop_group,
+                         chan_group=s.chan_group, n_pages=n // s.page_tokens, max_batch=1,
+                         max_pages_per_seq=n // s.page_tokens)
+    cb = codebooks_for_layer(s, 0, device=device, n_samples=1024, iters=10)[None].contiguous()
+    x = loop_group_kv(s, 0, 0, 0, n, device=device)
+    w = weights(s, n, True, device=device)
+    assign = torch.empty(L.loopvq_kmeans_assign_bytes(cfg, n), dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream()
+    L.loopvq_kmeans_step(cfg, 0, 0, 0, x, w, cb, assign, stream=st.cuda_stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(reps):
+        L.loopvq_kmeans_step(cfg, 0, 0, 0, x, w, cb, assign, stream=st.cuda_stream)
+    e1.record(st)
+    torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / reps
+    # the encoder alone on the same inputs: the step minus it is the update
+    pool = torch.zeros(L.loopvq_cache_layout(cfg)["pool_bytes"], dtype=torch.uint8, device=device)
+    cfg_e = cfg
+    slots = torch.arange(n, device=device, dtype=torch.int64)
+    L.loopvq_encode(cfg_e, 0, 0, 0, x, w, cb, slots, pool, stream=st.cuda_stream)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(reps):
+        L.loopvq_encode(cfg_e, 0, 0, 0, x, w, cb, slots, pool, stream=st.cuda_stream)
+    e1.record(st)
+    torch.cuda.synchronize()
+    enc_ms = e0.elapsed_time(e1) / reps
+    nsub = n * s.n_kv_heads * s.J
+    upd_ms = max(step_ms - enc_ms, 1e-6)
+    # update: x (bf16) and w (fp32) once, the assignment once, codebooks read and written
+    upd_bytes = n * s.n_kv_heads * s.head_dim * s.loop_group * (2 + 4) + nsub + \
+        2 * s.n_kv_heads * s.J * 256 * s.D * 4
+    return {"ms_per_step": step_ms, "subvectors_per_s": nsub / (step_ms / 1e3),
+            "assign_ms": enc_ms, "update_ms": upd_ms,
+            "update_gbps": upd_bytes / (upd_ms / 1e3) / 1e9, "update_bytes": upd_bytes,
+            "shape": f"{n} tokens x {s.n_kv_heads} heads x {s.J} groups, D={s.D}, "
+                     f"per-token LogNormal weights, one of K/V"}
+
+
 # --------------------------------------------------------------------------
 # main
 # --------------------------------------------------------------------------
@@ -567,6 +621,7 @@ def main():
         line["bf16_kv"] = bf16_comparison(shape, dev)
         line["bf16_kv"]["vq_speedup_per_call"] = line["bf16_kv"]["us_per_call"] / avg_call_us
         line["encode_prefill"] = encode_prefill(dev)
+        line["kmeans_step"] = kmeans_step(dev)
     if world > 1:
         import torch.distributed as dist
         barrier(world)

@@ -183,6 +183,38 @@ loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_
                             const int64_t* slot_mapping, uint8_t* pool, void* stream);
 
 /*
+ * One weighted k-means (Lloyd) step on the codebooks of (layer,
+ * loop_group_idx, K or V) for every kv-head and channel group: the offline
+ * codebook fitting that the abstract's quantiser needs (Fisher-weighted
+ * k-means, airadar.tv opening paragraph), run on the GPU.
+ *
+ * With the sub-vectors s and weights w of loopvq_encode (same x, w, strides
+ * and rules):
+ *   1. assignment: assign[(h*J + j)*n_tokens + n] = the index loopvq_encode
+ *      would write for token n under the current codebooks (same float32
+ *      arithmetic and tie rule);
+ *   2. update, in place: every element i of centroid e becomes
+ *          sum_{n: assign = e} w_ni s_ni / sum_{n: assign = e} w_ni,
+ *      the minimiser of the cluster's weighted squared distance; an element
+ *      whose weight sum is zero (an empty cluster, or zero weights) keeps its
+ *      value. The sums are float32 and their order is not fixed, so repeated
+ *      runs can differ in the last bits.
+ *
+ *  codebooks  base of the whole codebook array (layout above); read and
+ *             written.
+ *  assign     device buffer of at least loopvq_kmeans_assign_bytes(cfg,
+ *             n_tokens) bytes; receives the step's assignment.
+ * Returns LOOPVQ_ERR_WORKSPACE if assign_bytes is too small. n_tokens == 0
+ * is a no-op that returns LOOPVQ_OK.
+ */
+size_t loopvq_kmeans_assign_bytes(const loopvq_config* cfg, int n_tokens);
+loopvq_status loopvq_kmeans_step(const loopvq_config* cfg, int layer, int loop_group_idx, int kv,
+                                 int n_tokens, const void* x, int64_t x_loop_stride,
+                                 int64_t x_token_stride, const float* w, int64_t w_loop_stride,
+                                 int64_t w_token_stride, float* codebooks, uint8_t* assign,
+                                 size_t assign_bytes, void* stream);
+
+/*
  * Bytes of scratch that loopvq_decode_attn needs for `batch` sequences of
  * at most `max_seq_len` tokens: (batch*Hq + 256) segment records of
  * 4 + head_dim float32 (a segment's softmax maximum and sum and its

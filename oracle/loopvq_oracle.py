@@ -45,10 +45,11 @@ reason, in the design notes of the repository):
   against a dequantised key is a plain dot product.
 
 Pins (the tests under ``tests/test_oracle_*.py``) tie every function here to
-something other than itself: the rate closed form, scipy's ``vq`` and
-``logsumexp``, torch's ``scaled_dot_product_attention``, brute force over all
-assignments on tiny inputs, an exact codebook that must reproduce the
-unquantised cache, split-and-merge identities and invariances.
+something other than itself: the rate closed form, scipy's ``vq``,
+``kmeans2`` and ``logsumexp``, torch's ``scaled_dot_product_attention``,
+brute force over all assignments on tiny inputs, an exact codebook that must
+reproduce the unquantised cache, token replication for integer weights,
+split-and-merge identities and invariances.
 """
 
 from __future__ import annotations
@@ -196,6 +197,100 @@ def encode_group_ref(X: np.ndarray, cb: np.ndarray,
         idx[:, h] = i_h
         dist[:, h] = d_h
     return idx, dist
+
+
+# ---------------------------------------------------------------------------
+# Codebook fitting: one weighted k-means (Lloyd) step
+# ---------------------------------------------------------------------------
+# The codebooks are fitted offline with Fisher-weighted k-means (airadar.tv,
+# opening paragraph). A Lloyd step alternates the assignment (the encoder
+# above, under the current codewords) and the update. Under the per-element
+# weighted squared distance the update that minimises a cluster's distortion
+# is, element by element, the weighted mean of its members; an element with
+# no weight (an empty cluster) keeps its codeword value.
+
+def centroid_update_ref(S: np.ndarray, CW: np.ndarray, idx: np.ndarray,
+                        Wt: np.ndarray | None = None) -> np.ndarray:
+    """Weighted centroid update for the codebooks of one head, float64.
+
+    ``S`` is ``[N][J][D]``, ``CW`` the current codewords ``[J][E][D]``,
+    ``idx`` the assignment ``[N][J]``, ``Wt`` ``[N][J][D]`` or None (weight
+    1). Returns ``new[j, e, i] = sum_{n: idx[n,j]=e} Wt[n,j,i] S[n,j,i] /
+    sum_{n: idx[n,j]=e} Wt[n,j,i]``, or ``CW[j, e, i]`` where that weight sum
+    is zero.
+    """
+    S = np.asarray(S, dtype=np.float64)
+    CW = np.asarray(CW, dtype=np.float64)
+    idx = np.asarray(idx)
+    N, J, D = S.shape
+    W = np.ones_like(S) if Wt is None else np.asarray(Wt, dtype=np.float64)
+    new = CW.copy()
+    for j in range(J):
+        for e in range(CW.shape[1]):
+            members = idx[:, j] == e
+            if not members.any():
+                continue
+            den = W[members, j, :].sum(axis=0)
+            num = (W[members, j, :] * S[members, j, :]).sum(axis=0)
+            keep = den == 0
+            new[j, e] = np.where(keep, CW[j, e], num / np.where(keep, 1.0, den))
+    return new
+
+
+def codebook_from_codewords(CW: np.ndarray, g: int) -> np.ndarray:
+    """Inverse of ``codewords``: ``[J][E][g*c]`` back to ``[g][J][E][c]``."""
+    CW = np.asarray(CW, dtype=np.float64)
+    J, E, D = CW.shape
+    c = D // g
+    cb = np.empty((g, J, E, c), dtype=np.float64)
+    for tau in range(g):
+        cb[tau] = CW[:, :, tau * c:(tau + 1) * c]
+    return cb
+
+
+def kmeans_step_group_ref(X: np.ndarray, cb: np.ndarray, w: np.ndarray | None = None,
+                          assign: np.ndarray | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """One weighted Lloyd step on the per-head codebooks ``cb [H][g][J][E][c]``
+    of one loop group, with the g loop slices ``X [g][N][H][d]`` and weights
+    ``w`` as for ``encode_group_ref``.
+
+    The assignment is the encoder's under ``cb``, unless ``assign [N][H][J]``
+    is given (then that one is used, e.g. to update from another
+    implementation's choice among near-tied centroids). Returns
+    ``(assignment [N][H][J] uint8, new codebooks [H][g][J][E][c])``.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    g, N, H, d = X.shape
+    c = cb.shape[-1]
+    if assign is None:
+        assign, _ = encode_group_ref(X, cb, w)
+    S = subvectors(X, c)
+    Wt = subvector_weights(w, N, c)
+    new = np.empty(cb.shape, dtype=np.float64)
+    for h in range(H):
+        CW_new = centroid_update_ref(S[:, h], codewords(cb[h]), assign[:, h],
+                                     None if Wt is None else Wt[:, h])
+        new[h] = codebook_from_codewords(CW_new, g)
+    return np.asarray(assign, dtype=np.uint8), new
+
+
+def weighted_distortion_ref(X: np.ndarray, cb: np.ndarray, assign: np.ndarray,
+                            w: np.ndarray | None = None) -> float:
+    """Total weighted squared distance of every sub-vector to the codeword
+    it is assigned to (the objective a Lloyd step does not increase)."""
+    X = np.asarray(X, dtype=np.float64)
+    g, N, H, d = X.shape
+    c = cb.shape[-1]
+    S = subvectors(X, c)
+    Wt = subvector_weights(w, N, c)
+    total = 0.0
+    for h in range(H):
+        CW = codewords(cb[h])
+        for j in range(d // c):
+            diff = S[:, h, j, :] - CW[j][assign[:, h, j]]
+            sq = diff * diff if Wt is None else Wt[:, h, j, :] * diff * diff
+            total += float(sq.sum())
+    return total
 
 
 # ---------------------------------------------------------------------------

@@ -84,6 +84,10 @@ def _load() -> ctypes.CDLL:
     lib.loopvq_bf16_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.loopvq_bf16_decode_attn.restype = I
     lib.loopvq_bf16_decode_attn.argtypes = [I, I, I, I, I, P, P, P, P, F, I, P, P, P, SZ, P]
+    lib.loopvq_kmeans_assign_bytes.restype = SZ
+    lib.loopvq_kmeans_assign_bytes.argtypes = [cfgp, I]
+    lib.loopvq_kmeans_step.restype = I
+    lib.loopvq_kmeans_step.argtypes = [cfgp, I, I, I, I, P, I64, I64, P, I64, I64, P, P, SZ, P]
     return lib
 
 
@@ -91,7 +95,8 @@ _lib = _load()
 
 EXPORTED = ("loopvq_status_string", "loopvq_cache_layout", "loopvq_encode",
             "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
-            "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn")
+            "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn",
+            "loopvq_kmeans_assign_bytes", "loopvq_kmeans_step")
 
 
 def library() -> ctypes.CDLL:
@@ -183,6 +188,41 @@ def loopvq_encode(cfg: LoopVQConfig, layer: int, loop_group_idx: int, kv: int, x
                             x.stride(0), x.stride(1) if n > 1 else 0, _ptr(w), wl, wt,
                             _ptr(codebooks), _ptr(slot_mapping), _ptr(pool), _stream(stream))
     _check("loopvq_encode", st)
+
+
+def _xw_strides(x: torch.Tensor, w: torch.Tensor | None) -> tuple[int, int, int, int]:
+    n = x.shape[1]
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    if x.stride(3) != 1 or x.stride(2) != x.shape[3]:
+        raise ValueError("x rows [Hkv][d] must be dense")
+    wl = wt = 0
+    if w is not None:
+        if w.dtype != torch.float32 or w.stride(3) != 1 or w.stride(2) != w.shape[3]:
+            raise ValueError("w must be float32 with dense [Hkv][d] rows")
+        wl = w.stride(0)
+        wt = w.stride(1) if w.shape[1] != 1 else 0
+    return x.stride(0), (x.stride(1) if n > 1 else 0), wl, wt
+
+
+def loopvq_kmeans_assign_bytes(cfg: LoopVQConfig, n_tokens: int) -> int:
+    return int(_lib.loopvq_kmeans_assign_bytes(cfg.c_ref(), n_tokens))
+
+
+def loopvq_kmeans_step(cfg: LoopVQConfig, layer: int, loop_group_idx: int, kv: int, x: torch.Tensor,
+                       w: torch.Tensor | None, codebooks: torch.Tensor, assign: torch.Tensor,
+                       stream=None) -> None:
+    """One weighted Lloyd step on the codebooks of (layer, loop_group_idx,
+    kv), in place. x and w as for loopvq_encode; assign: uint8 with at least
+    loopvq_kmeans_assign_bytes(cfg, n) bytes, receives [Hkv][J][n]."""
+    n = x.shape[1]
+    xl, xt, wl, wt = _xw_strides(x, w)
+    if assign.dtype != torch.uint8:
+        raise TypeError("assign must be uint8")
+    st = _lib.loopvq_kmeans_step(cfg.c_ref(), layer, loop_group_idx, kv, n, _ptr(x), xl, xt,
+                                 _ptr(w), wl, wt, _ptr(codebooks), _ptr(assign),
+                                 assign.numel(), _stream(stream))
+    _check("loopvq_kmeans_step", st)
 
 
 def loopvq_decode_workspace_bytes(cfg: LoopVQConfig, batch: int, max_seq_len: int) -> int:

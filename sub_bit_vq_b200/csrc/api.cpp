@@ -198,8 +198,42 @@ loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_
   if (!loopvq::aligned(codebooks, 16) || !loopvq::aligned(slot_mapping, 8))
     return LOOPVQ_ERR_INVALID_ARG;
   loopvq::EncodeArgs a{&g, layer, loop_group_idx, kv, n_tokens, x, x_loop_stride, x_token_stride,
-                       w, w_loop_stride, w_token_stride, codebooks, slot_mapping, pool, stream};
+                       w, w_loop_stride, w_token_stride, codebooks, slot_mapping, pool, nullptr, stream};
   return loopvq::launch_encode(a);
+}
+
+size_t loopvq_kmeans_assign_bytes(const loopvq_config* cfg, int n_tokens) {
+  Geometry g;
+  if (loopvq::make_geometry(cfg, &g) != LOOPVQ_OK || n_tokens < 0) return 0;
+  return static_cast<size_t>(g.Hkv) * g.J * static_cast<size_t>(n_tokens);
+}
+
+loopvq_status loopvq_kmeans_step(const loopvq_config* cfg, int layer, int loop_group_idx, int kv,
+                                 int n_tokens, const void* x, int64_t x_loop_stride,
+                                 int64_t x_token_stride, const float* w, int64_t w_loop_stride,
+                                 int64_t w_token_stride, float* codebooks, uint8_t* assign,
+                                 size_t assign_bytes, void* stream) {
+  Geometry g;
+  loopvq_status st = loopvq::make_geometry(cfg, &g);
+  if (st != LOOPVQ_OK) return st;
+  if (layer < 0 || layer >= g.L || loop_group_idx < 0 || loop_group_idx >= g.G) return LOOPVQ_ERR_INVALID_ARG;
+  if (kv != 0 && kv != 1) return LOOPVQ_ERR_INVALID_ARG;
+  if (n_tokens < 0) return LOOPVQ_ERR_INVALID_ARG;
+  if (n_tokens == 0) return LOOPVQ_OK;
+  if (x == nullptr || codebooks == nullptr || assign == nullptr) return LOOPVQ_ERR_INVALID_ARG;
+  if (!loopvq::aligned(x, 16) || x_loop_stride < 0 || x_token_stride < 0 ||
+      (x_loop_stride % 8) != 0 || (x_token_stride % 8) != 0)
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (w != nullptr && (!loopvq::aligned(w, 16) || w_loop_stride < 0 || w_token_stride < 0 ||
+                       (w_loop_stride % 4) != 0 || (w_token_stride % 4) != 0))
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (!loopvq::aligned(codebooks, 16)) return LOOPVQ_ERR_INVALID_ARG;
+  if (assign_bytes < loopvq_kmeans_assign_bytes(cfg, n_tokens)) return LOOPVQ_ERR_WORKSPACE;
+  loopvq::EncodeArgs a{&g, layer, loop_group_idx, kv, n_tokens, x, x_loop_stride, x_token_stride,
+                       w, w_loop_stride, w_token_stride, codebooks, nullptr, nullptr, assign, stream};
+  st = loopvq::launch_encode(a);                       // assignment under the current codebooks
+  if (st != LOOPVQ_OK) return st;
+  return loopvq::launch_kmeans_update(a, codebooks);   // weighted means, in place
 }
 
 loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_step, int batch,

@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(kEncWarpThreads) encode_warp_kernel(const Enco
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int n = warp; n < p.n_tokens; n += kEncWarpThreads / 32) {
-    const int64_t slot = p.slot_mapping[n];
+    const int64_t slot = token_slot(p, n);
     if (slot < 0 || slot >= p.n_slots) continue;   // warp-uniform
     float s[D], w[D];
     load_subvector<C, G>(p, n, j, h, s, w);
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
   __syncthreads();
   const int n = blockIdx.x * kEncThreads + threadIdx.x;
   if (n >= p.n_tokens) return;
-  const int64_t slot = p.slot_mapping[n];
+  const int64_t slot = token_slot(p, n);
   if (slot < 0 || slot >= p.n_slots) return;
 
   float s[D], w[D];
@@ -140,7 +140,7 @@ loopvq_status launch_enc(const EncodeParams& p, int J, int H, cudaStream_t st) {
 
 }  // namespace
 
-loopvq_status launch_encode(const EncodeArgs& a) {
+EncodeParams encode_params(const EncodeArgs& a) {
   const Geometry& g = *a.geo;
   EncodeParams p{};
   p.x = static_cast<const uint16_t*>(a.x);
@@ -154,11 +154,13 @@ loopvq_status launch_encode(const EncodeArgs& a) {
   p.cb_stride_head = g.cb_stride_head;
   p.cb_stride_loop = g.cb_stride_loop;
   p.slot_mapping = a.slot_mapping;
-  p.pool = a.pool + a.layer * g.pool_stride_layer + a.gamma * g.pool_stride_group;
+  p.assign = a.assign;
+  p.pool = (a.pool != nullptr) ? a.pool + a.layer * g.pool_stride_layer + a.gamma * g.pool_stride_group
+                               : nullptr;
   p.pool_stride_head = g.pool_stride_head;
   p.page_bytes = g.page_bytes;
   p.plane_bytes = g.plane_bytes;
-  p.n_slots = static_cast<int64_t>(g.n_pages) * g.Pg;
+  p.n_slots = (a.assign != nullptr) ? a.n_tokens : static_cast<int64_t>(g.n_pages) * g.Pg;
   p.n_tokens = a.n_tokens;
   p.d = g.d;
   p.Pg = g.Pg;
@@ -166,6 +168,12 @@ loopvq_status launch_encode(const EncodeArgs& a) {
   p.LB = g.LB;
   p.GR = g.GR;
   p.kv = a.kv;
+  return p;
+}
+
+loopvq_status launch_encode(const EncodeArgs& a) {
+  const Geometry& g = *a.geo;
+  const EncodeParams p = encode_params(a);
   cudaStream_t st = static_cast<cudaStream_t>(a.stream);
   switch (g.c * 100 + g.g) {
     case 404: return launch_enc<4, 4>(p, g.J, g.Hkv, st);

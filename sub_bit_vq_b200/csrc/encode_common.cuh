@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "internal.h"
 #include "loopvq.h"
 
 namespace loopvq {
@@ -15,15 +16,26 @@ struct EncodeParams {
   int64_t w_loop_stride, w_token_stride;
   const float* cb;              // codebooks at (layer, head 0, gamma, kv, tau 0)
   int64_t cb_stride_head, cb_stride_loop;
-  const int64_t* slot_mapping;
+  const int64_t* slot_mapping;  // null: token n is slot n
   uint8_t* pool;                // pool at (layer, head 0, gamma)
+  uint8_t* assign;              // or null: indices [H][J][n_tokens] instead of the pool
   int64_t pool_stride_head, page_bytes, plane_bytes;
   int64_t n_slots;              // n_pages * Pg
   int n_tokens, d, Pg, J, LB, GR, kv;
 };
 
-// Writes index `e` of (slot, group j, head h) to its byte in the pool.
+// Slot of token n: its pool slot, or n itself when indices go to `assign`.
+__device__ __forceinline__ int64_t token_slot(const EncodeParams& p, int n) {
+  return p.slot_mapping != nullptr ? p.slot_mapping[n] : static_cast<int64_t>(n);
+}
+
+// Writes index `e` of (slot, group j, head h) to its byte in the pool, or to
+// assign[h][j][slot].
 __device__ __forceinline__ void store_index(const EncodeParams& p, int64_t slot, int j, int h, int e) {
+  if (p.assign != nullptr) {
+    p.assign[(static_cast<int64_t>(h) * p.J + j) * p.n_tokens + slot] = static_cast<uint8_t>(e);
+    return;
+  }
   const int64_t page = slot / p.Pg;
   const int sl = static_cast<int>(slot % p.Pg);
   int64_t off;
@@ -62,6 +74,9 @@ __device__ __forceinline__ void load_subvector(const EncodeParams& p, int n, int
     }
   }
 }
+
+// Kernel parameters of an encode (or k-means) call; see encode.cu.
+EncodeParams encode_params(const EncodeArgs& a);
 
 // Launches the tensor-core encoder (D = c*g in {8, 16, 32}); see encode_tc.cu.
 bool encode_tc_supported(int c, int g);

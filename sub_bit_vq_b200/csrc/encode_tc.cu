@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
   int64_t slot_nx = -1;
   auto fetch = [&](int t) {
     const int n = t * kTcRows + tid;
-    slot_nx = (t < n_tiles && n < p.n_tokens) ? p.slot_mapping[n] : -1;
+    slot_nx = (t < n_tiles && n < p.n_tokens) ? token_slot(p, n) : -1;
     if (slot_nx >= 0 && slot_nx < p.n_slots) load_subvector<C, G>(p, n, j, h, s_nx, w_nx);
   };
   fetch(0);

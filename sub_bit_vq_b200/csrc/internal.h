@@ -25,7 +25,7 @@ int max_decode_splits(int pairs, int pages);
 
 // Most CTAs the persistent LoopVQ streaming kernel is launched with (one per
 // SM up to this many); the decode workspace holds (pairs + kMaxStreamCtas)
-// segment records of 4 + 256*J floats.
+// segment records of 4 + d floats.
 constexpr int kMaxStreamCtas = 256;
 
 // Number of multiprocessors of the current device (cached per device).
@@ -61,11 +61,18 @@ struct EncodeArgs {
   const float* w;
   int64_t w_loop_stride, w_token_stride;
   const float* codebooks;
-  const int64_t* slot_mapping;
-  uint8_t* pool;
+  const int64_t* slot_mapping;   // null: token n is slot n of `assign`
+  uint8_t* pool;                 // null when `assign` is given
+  uint8_t* assign;               // or null: indices [Hkv][J][n_tokens] instead of the pool
   void* stream;
 };
 loopvq_status launch_encode(const EncodeArgs& a);
+
+// Weighted centroid update of one k-means step: every codebook (h, j) of
+// (layer, gamma, kv) becomes the per-element weighted mean of the
+// sub-vectors assigned to each centroid (assignment [Hkv][J][n_tokens]);
+// elements whose weight sum is zero keep their value.
+loopvq_status launch_kmeans_update(const EncodeArgs& a, float* codebooks);
 
 struct Bf16DecodeArgs {
   int batch, Hq, Hkv, d, max_seq_len;

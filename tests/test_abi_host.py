@@ -139,6 +139,35 @@ def test_encode_rejects_before_launch():
     assert enc(sm=0x4004) == E
 
 
+def test_kmeans_step_rejects_before_launch():
+    cfg = _cfg()
+    lib = B.library()
+    n = 10
+    need = L.loopvq_kmeans_assign_bytes(cfg, n)
+    assert need == 3 * (128 // 4) * n                 # Hkv * J * n_tokens
+    assert L.loopvq_kmeans_assign_bytes(cfg, -1) == 0
+
+    def km(layer=0, grp=0, kv=0, n=n, x=0x1000, xl=512, xt=1024, w=None, wl=0, wt=0, cb=0x3000,
+           assign=0x4000, nbytes=need):
+        return lib.loopvq_kmeans_step(ctypes.byref(cfg.c_struct()), layer, grp, kv, n, x, xl, xt, w,
+                                      wl, wt, cb, assign, nbytes, None)
+    E = B.LOOPVQ_ERR_INVALID_ARG
+    assert km(n=0, x=None, cb=None, assign=None, nbytes=0) == B.LOOPVQ_OK   # no-op
+    assert km(layer=2) == E
+    assert km(grp=2) == E
+    assert km(kv=2) == E
+    assert km(n=-1) == E
+    assert km(x=None) == E
+    assert km(cb=None) == E
+    assert km(assign=None) == E
+    assert km(x=0x1001) == E
+    assert km(xt=3) == E
+    assert km(w=0x2004) == E
+    assert km(w=0x2000, wt=3) == E
+    assert km(cb=0x3004) == E
+    assert km(nbytes=need - 1) == B.LOOPVQ_ERR_WORKSPACE
+
+
 def test_workspace_bytes_formula():
     cfg = _cfg()
     # one record (m, l, 2 spare, value histogram [256][J]) of float32 per

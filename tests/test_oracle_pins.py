@@ -381,3 +381,121 @@ def test_vector_packer_matches_scalar_packer(J):
         for kv in (0, 1):
             np.testing.assert_array_equal(O.plane_offsets(np.array([s]), J, kv, Pg)[0],
                                           [O.plane_offset(s, j, J, kv, Pg) for j in range(J)])
+
+
+# ---------------------------------------------------------------------------
+# Weighted k-means (Lloyd) step: scipy's kmeans2, token replication,
+# optimality of the update, descent of the objective
+# ---------------------------------------------------------------------------
+
+def _lloyd_case(seed, N=600, H=1, d=16, g=2, c=4, E=256, per_element=True):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((g, N, H, d))
+    cb = rng.standard_normal((H, g, d // c, E, c)) * 0.8
+    w = rng.lognormal(0.0, 1.0, (g, N, H, d)) if per_element else None
+    return X, cb, w
+
+
+def test_unweighted_lloyd_step_matches_scipy_kmeans2():
+    # one iteration of scipy's kmeans2 from a given code book is the same
+    # step: assignment by vq, then means, empty clusters kept in place
+    X, cb, _ = _lloyd_case(11, N=700, E=64)
+    idx, new = O.kmeans_step_group_ref(X, cb)
+    S = O.subvectors(X, 4)
+    CW = O.codewords(cb[0])
+    empty = 0
+    for j in range(S.shape[2]):
+        import warnings
+        with warnings.catch_warnings():
+            warnings.simplefilter("ignore")
+            ref_cb, ref_lab = scipy.cluster.vq.kmeans2(S[:, 0, j, :], CW[j].copy(), iter=1,
+                                                       minit="matrix")
+        np.testing.assert_array_equal(idx[:, 0, j], ref_lab)
+        np.testing.assert_allclose(O.codewords(new[0])[j], ref_cb, rtol=1e-12, atol=1e-12)
+        empty += int(np.sum(np.bincount(ref_lab, minlength=64) == 0))
+    assert empty > 0                       # the kept-in-place rule was exercised
+
+
+def test_integer_token_weights_equal_token_replication():
+    # a weight k on every element of a token is the token counted k times
+    X, cb, _ = _lloyd_case(12, N=300, E=32)
+    rng = np.random.default_rng(13)
+    k = rng.integers(1, 5, size=X.shape[1])
+    w = np.broadcast_to(k[None, :, None, None].astype(np.float64), X.shape).copy()
+    idx_w, new_w = O.kmeans_step_group_ref(X, cb, w)
+    Xr = np.repeat(X, k, axis=1)
+    idx_r, new_r = O.kmeans_step_group_ref(Xr, cb)
+    np.testing.assert_array_equal(np.repeat(idx_w, k, axis=0), idx_r)
+    np.testing.assert_allclose(new_w, new_r, rtol=1e-12, atol=1e-12)
+    S = O.subvectors(Xr, 4)
+    for j in range(S.shape[2]):
+        ref_cb, _ = scipy.cluster.vq.kmeans2(S[:, 0, j, :], O.codewords(cb[0])[j].copy(), iter=1,
+                                             minit="matrix", missing="warn")
+        np.testing.assert_allclose(O.codewords(new_w[0])[j], ref_cb, rtol=1e-12, atol=1e-12)
+
+
+def test_weighted_update_is_the_clusters_minimiser():
+    # for the given assignment, each updated element zeroes the gradient of
+    # the cluster's weighted distortion, and moving it only costs more
+    X, cb, w = _lloyd_case(14, N=500, E=16)
+    idx, new = O.kmeans_step_group_ref(X, cb, w)
+    S, Wt = O.subvectors(X, 4)[:, 0], O.subvector_weights(w, X.shape[1], 4)[:, 0]
+    CW = O.codewords(new[0])
+    rng = np.random.default_rng(15)
+    for j in range(S.shape[1]):
+        for e in np.unique(idx[:, 0, j]):
+            m = idx[:, 0, j] == e
+            grad = (Wt[m, j] * (CW[j, e] - S[m, j])).sum(axis=0)
+            assert np.max(np.abs(grad)) < 1e-9 * max(1.0, Wt[m, j].sum())
+            base = (Wt[m, j] * (S[m, j] - CW[j, e]) ** 2).sum()
+            for _ in range(3):
+                moved = CW[j, e] + rng.normal(0, 1e-3, CW.shape[2])
+                assert (Wt[m, j] * (S[m, j] - moved) ** 2).sum() > base
+
+
+def test_weight_scale_leaves_the_step_unchanged():
+    X, cb, w = _lloyd_case(16, N=400, E=32)
+    i1, n1 = O.kmeans_step_group_ref(X, cb, w)
+    i2, n2 = O.kmeans_step_group_ref(X, cb, w * 7.5)
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_allclose(n1, n2, rtol=1e-12, atol=1e-13)
+
+
+def test_lloyd_steps_never_increase_the_weighted_distortion():
+    X, cb, w = _lloyd_case(17, N=800, H=2, E=32)
+    idx, _ = O.encode_group_ref(X, cb, w)
+    prev = O.weighted_distortion_ref(X, cb, idx, w)
+    for _ in range(4):
+        idx, cb = O.kmeans_step_group_ref(X, cb, w)
+        after_update = O.weighted_distortion_ref(X, cb, idx, w)
+        assert after_update <= prev * (1 + 1e-12)
+        idx, _ = O.encode_group_ref(X, cb, w)
+        prev2 = O.weighted_distortion_ref(X, cb, idx, w)
+        assert prev2 <= after_update * (1 + 1e-12)
+        prev = prev2
+
+
+def test_empty_clusters_and_zero_weights_keep_their_codewords():
+    X, cb, w = _lloyd_case(18, N=50, E=256)
+    w[:, :, :, 0] = 0.0                    # element 0 of group 0 (channel 0, every loop) has no weight
+    idx, new = O.kmeans_step_group_ref(X, cb, w)
+    used = np.zeros((cb.shape[2], cb.shape[3]), dtype=bool)
+    for j in range(cb.shape[2]):
+        used[j, np.unique(idx[:, 0, j])] = True
+    assert (~used).sum() > 0
+    for j in range(cb.shape[2]):
+        np.testing.assert_array_equal(new[0, :, j][:, ~used[j]], cb[0, :, j][:, ~used[j]])
+    # channel 0 is element tau*c + 0 of group 0 for every tau: kept where weight-free
+    np.testing.assert_array_equal(new[0, :, 0, :, 0], cb[0, :, 0, :, 0])
+
+
+def test_update_with_a_given_assignment_uses_it():
+    X, cb, w = _lloyd_case(19, N=200, E=16)
+    rng = np.random.default_rng(20)
+    forced = rng.integers(0, 16, size=(X.shape[1], 1, 4)).astype(np.uint8)
+    idx, new = O.kmeans_step_group_ref(X, cb, w, assign=forced)
+    np.testing.assert_array_equal(idx, forced)
+    S, Wt = O.subvectors(X, 4)[:, 0], O.subvector_weights(w, X.shape[1], 4)[:, 0]
+    m = forced[:, 0, 2] == 5
+    want = (Wt[m, 2] * S[m, 2]).sum(0) / Wt[m, 2].sum(0)
+    np.testing.assert_allclose(O.codewords(new[0])[2, 5], want, rtol=1e-12)
