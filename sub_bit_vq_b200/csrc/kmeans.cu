@@ -11,7 +11,8 @@
 // weights) keeps its value.
 //
 // One CTA per codebook (channel group j, kv-head h): shared memory holds
-// num[e][i] and den[e][i]; the threads take tokens tid, tid + T, .. and add
+// num[e][i] and den[e][i] in rows of D + 1 floats (so that the lanes' rows
+// spread over the banks); the threads take tokens tid, tid + T, .. and add
 // each sub-vector into the row of its centroid with shared-memory float
 // atomics (so the float32 sums are order-dependent in their last bits); the
 // CTA then rewrites its codebook in place.
@@ -28,11 +29,12 @@ constexpr int kKmThreads = 256;
 template <int C, int G>
 __global__ void __launch_bounds__(kKmThreads) kmeans_update_kernel(const EncodeParams p, float* cb) {
   constexpr int D = C * G;
-  extern __shared__ float acc[];                       // num [E][D], then den [E][D]
+  constexpr int DP = D + 1;                            // padded row
+  extern __shared__ float acc[];                       // num [E][DP], then den [E][DP]
   float* num = acc;
-  float* den = acc + kE * D;
+  float* den = acc + kE * DP;
   const int j = blockIdx.x, h = blockIdx.y;
-  for (int i = threadIdx.x; i < 2 * kE * D; i += kKmThreads) acc[i] = 0.f;
+  for (int i = threadIdx.x; i < 2 * kE * DP; i += kKmThreads) acc[i] = 0.f;
   __syncthreads();
   const uint8_t* as = p.assign + (static_cast<int64_t>(h) * p.J + j) * p.n_tokens;
   for (int n = threadIdx.x; n < p.n_tokens; n += kKmThreads) {
@@ -41,8 +43,8 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_update_kernel(const EncodeP
     load_subvector<C, G>(p, n, j, h, s, w);
 #pragma unroll
     for (int i = 0; i < D; ++i) {
-      atomicAdd(num + e * D + i, w[i] * s[i]);
-      atomicAdd(den + e * D + i, w[i]);
+      atomicAdd(num + e * DP + i, w[i] * s[i]);
+      atomicAdd(den + e * DP + i, w[i]);
     }
   }
   __syncthreads();
@@ -50,14 +52,14 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_update_kernel(const EncodeP
   float* cbj = cb + h * p.cb_stride_head + static_cast<int64_t>(j) * kE * C;
   for (int k = threadIdx.x; k < kE * D; k += kKmThreads) {
     const int e = k / D, i = k % D;
-    const float dn = den[k];
-    if (dn > 0.f) cbj[(i / C) * p.cb_stride_loop + e * C + i % C] = num[k] / dn;
+    const float dn = den[e * DP + i];
+    if (dn > 0.f) cbj[(i / C) * p.cb_stride_loop + e * C + i % C] = num[e * DP + i] / dn;
   }
 }
 
 template <int C, int G>
 loopvq_status launch_update(const EncodeParams& p, float* cb, int J, int H, cudaStream_t st) {
-  constexpr size_t smem = 2u * kE * C * G * sizeof(float);
+  constexpr size_t smem = 2u * kE * (C * G + 1) * sizeof(float);
   static_assert(smem <= 227u * 1024u, "accumulators fit shared memory");
   if (smem > 48u * 1024u &&
       cudaFuncSetAttribute(kmeans_update_kernel<C, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
