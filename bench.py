@@ -411,7 +411,31 @@ def encode_prefill(device, reps=3):
     return {"subvectors_per_s": nsub / sec, "ms_per_call": sec * 1e3,
             "shape": f"{n} tokens x {s.n_kv_heads} heads x {s.J} groups, D={s.D}, "
                      f"per-token LogNormal weights, one of K/V",
-            "kernel": "tcgen05 split-bf16 contraction + exact float32 rescore (tensor cores)"}
+            "kernel": "tcgen05 split-bf16 contraction + exact float32 rescore (tensor cores)",
+            "bounds": encode_bounds(nsub, s.D, sec)}
+
+
+def encode_bounds(nsub: int, D: int, sec: float) -> dict:
+    """The encoder's three candidate bounds for nsub sub-vectors of D
+    elements with per-token weights, as fractions achieved in `sec`:
+    - hbm: bf16 x and float32 w read, one index byte written;
+    - tensor: the cross and weight terms of the distance, 2 * (2 D) * 256
+      flops per sub-vector (the algorithmic count; the split-bf16 operands
+      triple the issued work), against the measured bf16 GEMM rate;
+    - alu: 256 candidates x 3 operations (bias add, compare, select) per
+      sub-vector, against 148 SMs x 128 float32 lanes x the maximum SM clock."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    d = json.load(open(p)) if os.path.exists(p) else {}
+    hbm = float(d.get("hbm_gbs", FALLBACK_HBM_GBS)) * 1e9
+    tflops = float(d.get("bf16_tflops", 1590.0)) * 1e12
+    mhz = float(d.get("sm_max_mhz", 1965.0)) * 1e6
+    byt = nsub * (D * 2 + D * 4 + 1)
+    flop = nsub * 2 * (2 * D) * 256
+    alu = nsub * 256 * 3
+    alu_peak = 148 * 128 * mhz
+    return {"hbm_frac": byt / sec / hbm, "tensor_frac": flop / sec / tflops,
+            "alu_frac": alu / sec / alu_peak, "bytes": byt, "flops": flop, "alu_ops": alu,
+            "peaks": "MEASURED_PEAKS.json hbm_gbs and bf16_tflops; alu from 148 x 128 lanes x sm_max_mhz"}
 
 
 def kmeans_step(device, reps=3):

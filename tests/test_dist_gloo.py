@@ -74,3 +74,14 @@ def test_reference_arm_runs_on_rank_zero_only():
                        text=True, timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_encoder_bound_fractions():
+    import bench
+    b1 = bench.encode_bounds(1000, 16, 1e-3)
+    assert b1["bytes"] == 1000 * (16 * 2 + 16 * 4 + 1)
+    assert b1["flops"] == 1000 * 2 * 32 * 256
+    assert b1["alu_ops"] == 1000 * 256 * 3
+    b2 = bench.encode_bounds(1000, 16, 2e-3)
+    for k in ("hbm_frac", "tensor_frac", "alu_frac"):
+        assert abs(b2[k] * 2 - b1[k]) < 1e-12 * b1[k]
