@@ -167,6 +167,15 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def call_percentiles(times: list[float]) -> list[float]:
+    """p10, median and p90 of per-call times (nearest rank on the sorted list)."""
+    t = sorted(times)
+    if not t:
+        return [float("nan")] * 3
+    pick = lambda q: t[min(len(t) - 1, max(0, int(round(q * (len(t) - 1)))))]
+    return [pick(0.1), pick(0.5), pick(0.9)]
+
+
 def recorded_traffic(kernel_src: str, key: str):
     """dram bytes per launch from the committed ncu summary, if it was taken
     on the current source of the kernel; else None."""
@@ -619,6 +628,7 @@ def main():
                 peak_src == "measured" else "fallback 6650 GB/s",
                 "kernel": "vq_stream_kernel + vq_finish_kernel (per-call events)",
                 "algorithmic_bytes_per_launch": alg, "avg_launch_us": avg_call_us,
+                "launch_us_p10_median_p90": call_percentiles(call_us),
                 "frac_of_8tbs": achieved / 8000.0}
 
     line = {"metric": METRIC, "value": value, "unit": "µs/loop-step", "n_gpus": world,

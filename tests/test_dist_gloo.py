@@ -85,3 +85,10 @@ def test_encoder_bound_fractions():
     b2 = bench.encode_bounds(1000, 16, 2e-3)
     for k in ("hbm_frac", "tensor_frac", "alu_frac"):
         assert abs(b2[k] * 2 - b1[k]) < 1e-12 * b1[k]
+
+
+def test_call_percentiles():
+    import bench
+    assert bench.call_percentiles(list(range(11))) == [1, 5, 9]
+    assert bench.call_percentiles([3.0]) == [3.0, 3.0, 3.0]
+    assert all(v != v for v in bench.call_percentiles([]))      # NaN
