@@ -499,3 +499,13 @@ def test_update_with_a_given_assignment_uses_it():
     m = forced[:, 0, 2] == 5
     want = (Wt[m, 2] * S[m, 2]).sum(0) / Wt[m, 2].sum(0)
     np.testing.assert_allclose(O.codewords(new[0])[2, 5], want, rtol=1e-12)
+
+
+def test_lloyd_step_shared_weights_equal_repeated_per_token_weights():
+    # a weight vector shared over tokens ([g][1][H][d]) is the same vector given to every token
+    X, cb, w = _lloyd_case(21, N=300, H=2, E=32)
+    shared = w[:, :1]
+    i1, n1 = O.kmeans_step_group_ref(X, cb, shared)
+    i2, n2 = O.kmeans_step_group_ref(X, cb, np.repeat(shared, X.shape[1], axis=1))
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_allclose(n1, n2, rtol=0, atol=0)
