@@ -184,3 +184,15 @@ def test_status_strings():
     for s in range(5):
         assert L.loopvq_status_string(s)
     assert "unknown" in L.loopvq_status_string(99)
+
+
+def test_python_api_exports_the_documented_calls():
+    for name in ("LoopVQConfig", "loopvq_cache_layout", "loopvq_encode", "loopvq_kmeans_assign_bytes",
+                 "loopvq_kmeans_step", "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
+                 "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn",
+                 "loopvq_status_string"):
+        assert callable(getattr(L, name)), name
+    cfg = _cfg()
+    lay = L.loopvq_cache_layout(cfg)
+    assert lay["bits_per_element"] == 0.5
+    assert L.loopvq_kmeans_assign_bytes(cfg, 7) == 3 * 32 * 7
