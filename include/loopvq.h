@@ -85,21 +85,19 @@ typedef struct {
  * with one plane = Pg*J bytes holding the K (or V) indices of Pg token
  * slots.
  *
- * K plane: slots come in blocks of LB = floor(32/J)*J. Inside a block the
- * bytes are stored in granules of GR bytes (GR = 16 if J % 16 == 0, else 8
- * if J % 8 == 0, else 4) as
+ * Both planes (K and V) share one layout. Slots come in blocks of
+ * LB = floor(32/J)*J. Inside a block the bytes are stored in granules of GR
+ * bytes (GR = 16 if J % 16 == 0, else 8 if J % 8 == 0, else 4) as
  *     [J/GR granules][LB slots][GR bytes],
  * and the J index bytes of slot i are rotated: the index of channel group
  * j sits at byte position (j - (i mod LB)) mod J of that slot's row. So
- * the byte offset of (slot i, group j) inside the K plane is
+ * the byte offset of (slot i, group j) inside a plane is
  *     (i/LB)*LB*J + (pos/GR)*LB*GR + (i%LB)*GR + pos%GR,
  *     pos = (j - i%LB) mod J.
  * The rotation lets one warp lane per slot read its own row while the
- * lanes of a warp touch distinct columns of a [E][32] table, which keeps
- * shared memory free of bank conflicts.
- *
- * V plane: group-major, the byte of (slot i, group j) is at j*Pg + i. One
- * lane per channel group then owns one column of the value histogram.
+ * lanes of a warp touch distinct columns of a [E][32] table (the key
+ * lookup table, the value histogram), which keeps shared memory free of
+ * bank conflicts, and the granules make a warp's row loads contiguous.
  *
  * Quantised token v of a sequence (v = position - P, for positions
  * P .. N-R-1) lives in page block_table[b][v / Pg], slot v % Pg.
@@ -276,8 +274,12 @@ loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_s
  * launches nothing.
  *
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any
- * stream capture. All calls on a device share the one array and it keeps
+ * device, with that device current) and the library remembers it for the
+ * rest of the process; make that first call before any stream capture. The
+ * remembered address belongs to the device's primary context: after
+ * cudaDeviceReset, or anything else that destroys and recreates that
+ * context, it is stale, and calling this entry point again in the same
+ * process is not supported. All calls on a device share the one array and it keeps
  * the last call's contents (no initial contents are needed); calls whose
  * kernels overlap on the GPU, e.g. on two streams without ordering, race
  * on it and give undefined results.

@@ -400,13 +400,12 @@ def decode_attn_ref(q: np.ndarray, win_K: np.ndarray, win_V: np.ndarray,
 # library's own code. The pool is
 #     [n_layers][n_kv_heads][n_loop_groups][n_pages][2 (K, V)][plane]
 # with a plane of page_tokens * J bytes.
-# K plane: token slots come in blocks of LB = floor(32/J)*J. Inside a block,
-# bytes are grouped in granules of GR bytes (GR = 16 if J % 16 == 0, else 8
-# if J % 8 == 0, else 4) laid out
+# Both planes (K and V) share one layout: token slots come in blocks of
+# LB = floor(32/J)*J. Inside a block, bytes are grouped in granules of GR
+# bytes (GR = 16 if J % 16 == 0, else 8 if J % 8 == 0, else 4) laid out
 #     [J / GR granules][LB slots][GR bytes],
 # and the J index bytes of slot i are rotated: group j sits at byte position
 # (j - (i mod LB)) mod J of that slot's row.
-# V plane: group-major, (slot i, group j) at byte j * page_tokens + i.
 
 def pool_granule(J: int) -> int:
     if J % 16 == 0:
@@ -426,10 +425,9 @@ def rotation_block(J: int) -> int:
 
 
 def plane_offset(slot: int, j: int, J: int, kv: int = 0, page_tokens: int = 0) -> int:
-    """Byte offset of group ``j`` of token slot ``slot`` inside the K plane
-    (``kv = 0``) or the V plane (``kv = 1``, needs ``page_tokens``)."""
-    if kv == 1:
-        return j * page_tokens + slot
+    """Byte offset of group ``j`` of token slot ``slot`` inside a plane. The
+    K plane (``kv = 0``) and the V plane (``kv = 1``) share the layout;
+    ``kv`` and ``page_tokens`` are accepted for the callers' convenience."""
     gr = pool_granule(J)
     lb = rotation_block(J)
     blk, rot = divmod(slot, lb)
@@ -459,8 +457,6 @@ def plane_offsets(slots: np.ndarray, J: int, kv: int = 0, page_tokens: int = 0) 
     """Array form of ``plane_offset``: ``[n]`` slots -> ``[n][J]`` offsets."""
     slots = np.asarray(slots, dtype=np.int64)[:, None]
     j = np.arange(J, dtype=np.int64)[None, :]
-    if kv == 1:
-        return j * page_tokens + slots
     gr = pool_granule(J)
     lb = rotation_block(J)
     blk, rot = slots // lb, slots % lb

@@ -8,11 +8,13 @@ from .binding import (  # noqa: F401
     LOOPVQ_DTYPE_BF16,
     LOOPVQ_DTYPE_F32,
     LoopVQConfig,
+    LOOPVQ_STATIC_SCRATCH_BYTES,
     LoopVQError,
     loopvq_bf16_decode_attn,
     loopvq_bf16_decode_workspace_bytes,
     loopvq_cache_layout,
     loopvq_decode_attn,
+    loopvq_decode_attn_noalloc,
     loopvq_decode_workspace_bytes,
     loopvq_encode,
     loopvq_kmeans_assign_bytes,

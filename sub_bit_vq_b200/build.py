@@ -51,8 +51,6 @@ def _sources() -> list[str]:
 
 def _compile(src: str, obj: str, extra: list[str]) -> None:
     cmd = [_nvcc(), "-c", src, "-o", obj] + NVCC_FLAGS + extra
-    if src.endswith(".cpp"):
-        cmd += ["-x", "cu"] if False else []
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{r.stdout}\n{r.stderr}")

@@ -171,7 +171,7 @@ size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int ma
   // (pair, streaming CTA) segment: record slots pair + cta never collide, so
   // pairs + CTAs slots suffice
   const size_t slots = static_cast<size_t>(batch) * g.Hq + loopvq::kMaxStreamCtas;
-  return slots * (4 + static_cast<size_t>(g.d)) * sizeof(float);
+  return loopvq::kStatusBytes + slots * (4 + static_cast<size_t>(g.d)) * sizeof(float);
 }
 
 loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_idx, int kv,

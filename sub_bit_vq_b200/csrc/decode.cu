@@ -2,50 +2,51 @@
 //
 // Two kernels per call.
 //
-// vq_stream_kernel: a persistent grid (at most one CTA per SM, twelve warps)
+// vq_stream_kernel: a persistent grid (at most one CTA per SM, sixteen warps)
 // over the quantised tokens of every (sequence, query head) pair. All pages
 // of all pairs form one list and CTA c takes the contiguous range
 // [U*c/n, U*(c+1)/n) of it, so every CTA streams the same number of pages and
 // touches one or a few pairs ("segments"). Per segment:
 //   1. The key codebook slice of the pair's kv-head and loop step is staged
-//      into the (empty) histogram windows with cp.async while the warps
+//      into the (empty) histogram window with cp.async while the warps
 //      request their first index blocks (a register ring); the key lookup
 //      table LUT[e][col] = s*log2(e) * q_j . C_K[j][e][tau] (column col holds
-//      group j = col % J) is built from it and the windows are zeroed.
-//   2. Streaming. Warp w takes pages w, w+12, ...; a block is LB token slots
-//      (LB = floor(32/J)*J), two blocks per round. Key pass: lane = slot;
-//      byte s of the slot's rotated row is group (lane+s) % J, held by LUT
-//      column (lane+s) % LB. Value pass: the weights p = 2^(x - m) are added
-//      into a histogram W[e][col]: lane = (replica, group) owns column
-//      `lane`, rows come from the group-major value bytes, four slots at a
-//      time; a weight whose row repeats later among the four is folded into
-//      that later update, so the last store of a row carries all of them.
-//      Three warps (w, w+4, w+8: one scheduler) share a histogram and take
-//      turns through bounded mbarrier waits; a warp computes its key scores
-//      and weights before its turn and only the histogram updates inside it.
-//      Each histogram keeps one running maximum m, raised only when a vote
-//      finds a score above m + kRescaleSlack.
-//   3. The four histograms are merged with log-sum-exp weights into W[E][J],
-//      which is contracted with the value codebook slice,
-//      o_j = sum_e W[e][j] C_V[j][e][tau]; the segment record (m, l, o[d]) goes
-//      to slot (pair + cta).
+//      group j = col % J) is built from it and the window is zeroed.
+//   2. Streaming, in chunks of kChunkBlocks blocks per warp. Key phase:
+//      lane = slot; byte s of the slot's rotated row is group (lane+s) % J,
+//      held by LUT column lane+s (the LUT repeats its J columns over 64), and
+//      the scores x (log2 units) stay in registers.
+//      The warps' maxima meet at a barrier; the segment's reference maximum
+//      m becomes the integer ceil(max x) so far (when it rises, the histogram
+//      is shifted right by the difference, which is exact in fixed point).
+//      Value phase, lane = slot again: the slot's weight 2^(x - m) <= 1
+//      becomes the integer w = rn(2^(x - m) * 2^kFixBits) and is added, for
+//      each byte s of the slot's rotated value row, to the shared histogram
+//      cell H[idx][(lane + s) % LB] by a 32-bit shared-memory atomic add on
+//      the low word of a 64-bit cell, with the carry added to the high word.
+//      Integer atomics run at full shared-memory rate on sm_100 and need no
+//      turn taking, so all warps update the one histogram concurrently.
+//   3. The histogram, converted to float, is contracted with the value
+//      codebook slice, o_j = sum_e W[e][j] C_V[j][e][tau], and the segment
+//      record (m, l = sum_e W[e][j], o[d]) goes to slot (pair + cta).
 //
 // vq_finish_kernel: one CTA per pair scores the bf16 window tokens (prefix +
 // recent), merges them with the pair's segment records (log-sum-exp
 // weights) and writes out and lse.
 //
 // The hot loops address shared memory by absolute shared-window address, so
-// that one byte permute of an index word gives a complete address: the
-// histograms occupy the 64 KB-aligned windows [0x10000, 0x30000) (row e at
-// byte e*256 of its window, two histograms per window) and the LUT the
-// window [0x8000, 0x10000) with 128-byte rows. The dynamic allocation starts
-// at a small base (the CTA's reserved bytes) and is sized to cover both; a
-// CTA whose base leaves no room below the LUT writes NaN records instead of
+// that one byte permute of an index byte gives a complete address: the LUT
+// sits in a 64 KB-aligned window with 256-byte rows (64 columns) and the
+// histogram in the next 64 KB window with 256-byte rows (low words in bytes
+// 0..127 of a row, high words in bytes 128..255). Both windows are placed at run time
+// above the dynamic allocation's base; a CTA whose allocation cannot hold
+// them writes NaN records and flags the call's status word instead of
 // running.
 
 #include <math.h>
 
 #include <atomic>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -53,31 +54,40 @@
 namespace loopvq {
 namespace {
 
-constexpr int kNHist = 4;                 // value histograms
-constexpr int kPerHist = 3;               // warps taking turns on one histogram
-constexpr int kNW = kNHist * kPerHist;    // warps of the streaming kernel
+constexpr int kNW = 16;                   // warps of the streaming kernel
 constexpr int kThreads = kNW * 32;
-constexpr int kRing = kPerHist >= 3 ? 2 : 4;   // index blocks in registers (rounds of two ahead)
-constexpr int kPrefetchPages = 8;         // pages a warp asks L2 to fetch ahead of its loads
-constexpr float kRescaleSlack = 8.0f;     // log2 units a score may exceed m before m is raised
+constexpr int kRing = 4;                  // index blocks in registers
+constexpr int kChunkBlocks = 4;           // blocks per warp per chunk (key phase, then value phase)
+constexpr int kPrefetchPages = 4;         // pages a warp asks L2 to fetch ahead of its loads
+constexpr int kFixBits = 30;              // fixed-point weight: w = rn(p * 2^kFixBits), p <= 1
+constexpr float kFixScale = 1073741824.0f;          // 2^kFixBits
+constexpr float kFixInv = 1.0f / 1073741824.0f;     // 2^-kFixBits
 constexpr int kFinishThreads = 256;
 constexpr int kWinChunk = 9;              // window tokens per warp per round of loads (72 = 8 warps x 9)
-constexpr int kSegmentUnits = 16;        // work units (pages) charged for a segment's setup
-constexpr int kSpinLimit = 1 << 14;       // bounded mbarrier waits (each try sleeps up to kSuspendNs)
-constexpr uint32_t kSuspendNs = 65536u;
-
-constexpr uint32_t kLutAbs = 0x8000u;     // LUT [E][32] floats, 128-byte rows
-constexpr uint32_t kHistAbs = 0x10000u;   // histogram h: window 1 + h/2, bytes (h%2)*128 .. of each row
-constexpr uint32_t kHistEnd = 0x30000u;   // (the key slice is staged here before a segment streams)
-constexpr uint32_t kDynBytes = kHistEnd;  // covers every window from any base >= 0
+constexpr int kSegmentUnits = 16;         // work units (pages) charged for a segment's setup
 
 // Small area at the start of the dynamic allocation (byte offsets).
-constexpr uint32_t kPbufOff = 0;                                  // [kNW][64] slot weights
-constexpr uint32_t kWstatOff = kPbufOff + kNW * 64 * 4;           // [2*kNW] per-warp m, l
-constexpr uint32_t kHmOff = kWstatOff + 2 * kNW * 4;              // [kNHist] running maxima
-constexpr uint32_t kFlagOff = kHmOff + kNHist * 4;                // [4] ints
-constexpr uint32_t kMbarOff = (kFlagOff + 16 + 7) & ~7u;          // [kNHist][kPerHist] mbarriers
-constexpr uint32_t kSmallBytes = kMbarOff + kNHist * kPerHist * 8;
+constexpr uint32_t kWmaxOff = 0;                                  // [2][kNW] chunk maxima
+constexpr uint32_t kQsOff = kWmaxOff + 2 * kNW * 4;               // [256] scaled q
+constexpr uint32_t kSmallBytes = kQsOff + 256 * 4;
+constexpr uint32_t kLutBytes = 0x10000u;  // [E][64] floats: column c holds group c % J
+constexpr uint32_t kHistBytes = 0x10000u; // [E][64] words: 32 low, 32 high
+// From any base b with b + kSmallBytes <= 0x10000 the LUT window starts at
+// 0x10000 and the histogram window at 0x20000, so the allocation must reach
+// 0x30000 - b; asking for 0x30000 bytes covers every such base.
+constexpr uint32_t kDynBytes = 0x30000u;
+
+// Groups of a [J][E][C] float codebook slice staged at once into the
+// histogram window: the largest divisor of J whose slice part fits.
+constexpr int stage_groups(int J, int C) {
+  int jc = J;
+  while (jc > 1 && (J % jc != 0 || jc * 256 * C * 4 > static_cast<int>(kHistBytes))) --jc;
+  return jc;
+}
+
+// Bits of the status word (see loopvq.h).
+constexpr int kStatusBadPage = 1;
+constexpr int kStatusSharedBase = 2;
 
 struct DecodeParams {
   const uint16_t* q;                // bf16 bits [B][Hq][d]
@@ -91,6 +101,7 @@ struct DecodeParams {
   const uint16_t* win_k;            // bf16 bits [B][Hkv][W][d]
   const uint16_t* win_v;
   float* records;                   // [pairs + n_cta][4 + d]: m, l, -, -, o[d]
+  int* status;                      // status word (bit flags), never cleared by the kernels
   void* out;
   float* lse;
   int B, Hq, Hkv, ratio, W, Pg, n_pages, max_pages_per_seq, max_seq_len;
@@ -104,13 +115,14 @@ struct Traits {
   static constexpr int R = 32 / J;      // replicas of each group per block
   static constexpr int LB = R * J;      // slots per block
   static constexpr int GR = (J % 16 == 0) ? 16 : (J % 8 == 0) ? 8 : 4;   // granule
-  static constexpr int NWORD = J / 4;   // words per lane per plane and block
+  static constexpr int NWORD = J / 4;   // words per lane and block
 };
 
+// One index block in registers: the rotated row of slot `lane` of the K
+// plane (a key item) or of the V plane (a value item).
 template <int J>
 struct BlockRegs {
-  uint32_t k[J / 4];   // this lane's rotated key row (lane = slot)
-  uint32_t v[J / 4];   // this lane's value bytes: group j, J consecutive slots
+  uint32_t w[J / 4];
   int base;            // first slot of the block inside its page, or -1: no block
   int valid;           // valid slots in the page (same value in every lane)
 };
@@ -131,25 +143,20 @@ __device__ __forceinline__ void load_words(const uint8_t* src, uint32_t* w, int 
   }
 }
 
-// Loads block `blk` of the page at `kpl` (K plane; the V plane follows).
+// Loads block `blk` of a page's K plane (kv = 0) or V plane (kv = 1): both
+// planes hold rotated slot rows in granules, so lane = slot reads its row.
 template <int J>
-__device__ __forceinline__ void load_block(const uint8_t* kpl, int64_t plane_bytes, int Pg, int blk,
+__device__ __forceinline__ void load_block(const uint8_t* kpl, int64_t plane_bytes, int blk, int kv,
                                            int lane, BlockRegs<J>& r) {
   using T = Traits<J>;
   if (lane < T::LB) {
+    const uint8_t* src = kpl + kv * plane_bytes + blk * T::LB * J + lane * T::GR;
 #pragma unroll
     for (int gi = 0; gi < J / T::GR; ++gi)
-      load_words<T::GR>(kpl + blk * T::LB * J + gi * T::LB * T::GR + lane * T::GR,
-                        r.k + gi * (T::GR / 4), T::GR / 4);
-    const int rr = lane / J, j = lane % J;
-    load_words<T::GR>(kpl + plane_bytes + static_cast<int64_t>(j) * Pg + blk * T::LB + rr * J, r.v,
-                      T::NWORD);
+      load_words<T::GR>(src + gi * T::LB * T::GR, r.w + gi * (T::GR / 4), T::GR / 4);
   } else {
 #pragma unroll
-    for (int i = 0; i < T::NWORD; ++i) {
-      r.k[i] = 0u;
-      r.v[i] = 0u;
-    }
+    for (int i = 0; i < T::NWORD; ++i) r.w[i] = 0u;
   }
 }
 
@@ -194,54 +201,63 @@ __device__ __forceinline__ float dot_c(const float* a, const float* b) {
   return v;
 }
 
+// Calls f(std::integral_constant<int, i>) for i = 0 .. N-1 (compile-time i).
+template <int N, typename F, int... I>
+__device__ __forceinline__ void constexpr_for_impl(F&& f, std::integer_sequence<int, I...>) {
+  (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void constexpr_for(F&& f) {
+  constexpr_for_impl<N>(f, std::make_integer_sequence<int, N>{});
+}
+
 // ---- shared memory by absolute shared-window address ------------------------
 
 __device__ __forceinline__ uint32_t smem_addr(const void* ptr) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
 }
 
-// Histogram words: ordered among themselves and against other memory
-// accesses (read-modify-write chains depend on it).
-__device__ __forceinline__ float lds_h(uint32_t a) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ void sts_h(uint32_t a, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
-}
-// LUT words: not written while they are read, so no ordering against stores.
+// LUT word at address a + OFF: not written while it is read.
+template <int OFF>
 __device__ __forceinline__ float lds_lut(uint32_t a) {
   float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(OFF));
   return v;
 }
-
-__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t a) {
-  asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(a) : "memory");
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
-  uint32_t done;
+// Histogram update: low word += w; on a carry out of the low word, the high
+// word (128 bytes further along the row) += 1.
+// Histogram updates of four cells by the same weight w: the low words at
+// a0..a3 get w added and their old values come back in o0..o3.
+__device__ __forceinline__ void hist_add4(const uint32_t (&a)[4], uint32_t w, uint32_t (&o)[4]) {
   asm volatile(
-      "{\n .reg .pred P;\n mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n"
-      " selp.u32 %0, 1, 0, P;\n}\n"
-      : "=r"(done)
-      : "r"(a), "r"(parity), "n"(kSuspendNs)
-      : "memory");
-  return done != 0u;
+      "atom.shared.add.u32 %0, [%4], %8;\n"
+      "atom.shared.add.u32 %1, [%5], %8;\n"
+      "atom.shared.add.u32 %2, [%6], %8;\n"
+      "atom.shared.add.u32 %3, [%7], %8;\n"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(w));
 }
-// Waits for the phase of parity `parity` to complete (each try sleeps until
-// the phase completes or kSuspendNs pass); gives up (false) after kSpinLimit
-// tries instead of hanging.
-__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
-  for (int i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(a, parity)) return true;
-    __nanosleep(64);                                   // leave the issue slots to the working warps
-  }
-  return false;
+// The carries of those four updates: where an old low word exceeded
+// nw = ~w (the sum wrapped), the high word 128 bytes further along the row
+// gets 1.
+__device__ __forceinline__ void hist_carry4(const uint32_t (&a)[4], const uint32_t (&o)[4],
+                                            uint32_t nw) {
+  asm volatile(
+      "{\n .reg .pred P<4>;\n"
+      " setp.gt.u32 P0, %4, %8;\n setp.gt.u32 P1, %5, %8;\n"
+      " setp.gt.u32 P2, %6, %8;\n setp.gt.u32 P3, %7, %8;\n"
+      " @P0 red.shared.add.u32 [%0+128], 1;\n @P1 red.shared.add.u32 [%1+128], 1;\n"
+      " @P2 red.shared.add.u32 [%2+128], 1;\n @P3 red.shared.add.u32 [%3+128], 1;\n}\n"
+      ::"r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]),
+      "r"(nw));
 }
 
 // Quantised-token pages of sequence b.
@@ -409,47 +425,43 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
   __syncthreads();
 }
 
+
 template <int J, int C>
 __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodeParams p) {
   using T = Traits<J>;
   constexpr int d = J * C;
   constexpr int LB = T::LB;
+  constexpr int KB = kChunkBlocks;                     // blocks per warp per chunk
   constexpr int RS = 4 + d;                            // record floats
   constexpr int EP = kE + 1;                           // padded row of the transposed merged histogram
-  static_assert(J * EP * 4 <= static_cast<int>(kHistEnd - kHistAbs), "merged histogram fits the windows");
-  // groups of the key slice staged at once in the (empty) histogram windows
-  constexpr int JC = (J * kE * C * 4 <= static_cast<int>(kHistEnd - kHistAbs))
-                         ? J : static_cast<int>(kHistEnd - kHistAbs) / (kE * C * 4);
-  static_assert(J % JC == 0, "staging chunks tile the groups");
-  static_assert(d <= kNW * 64 && d <= kThreads, "q fits the weight buffer");
+  static_assert(J * EP * 4 <= static_cast<int>(kHistBytes), "merged histogram fits the window");
+  static_assert((2 * KB) % kRing == 0, "a chunk's items map onto fixed ring slots");
+  // groups of the key slice staged at once in the (empty) histogram window
+  constexpr int JC = stage_groups(J, C);
+  static_assert(JC >= 1 && J % JC == 0, "staging chunks tile the groups");
+  static_assert(d <= 256, "q fits its buffer");
 
   extern __shared__ __align__(16) unsigned char smem_u8[];
   const uint32_t sbase = smem_addr(smem_u8);
-  float* pbuf = reinterpret_cast<float*>(smem_u8 + kPbufOff);
-  float* wstat = reinterpret_cast<float*>(smem_u8 + kWstatOff);
-  float* hm = reinterpret_cast<float*>(smem_u8 + kHmOff);
-  int* flags = reinterpret_cast<int*>(smem_u8 + kFlagOff);
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem_u8 + kMbarOff);
-  // a base that leaves no room below the LUT window: poison records, do nothing else
-  const bool bad_base = sbase + kSmallBytes > kLutAbs;
-  float* lut = reinterpret_cast<float*>(smem_u8 + (bad_base ? 0u : kLutAbs - sbase));
-  float* stage = reinterpret_cast<float*>(smem_u8 + (bad_base ? 0u : kHistAbs - sbase));
-  float* qs = pbuf;                                    // scaled q while the LUT is built
+  float* wmax = reinterpret_cast<float*>(smem_u8 + kWmaxOff);
+  float* qs = reinterpret_cast<float*>(smem_u8 + kQsOff);
+  // the LUT and histogram windows, aligned above the small area
+  const uint32_t lut_abs = (sbase + kSmallBytes + kLutBytes - 1u) & ~(kLutBytes - 1u);
+  const uint32_t hist_abs = lut_abs + kLutBytes;
+  const bool bad_base = hist_abs + kHistBytes > sbase + kDynBytes;
+  float* lut = reinterpret_cast<float*>(smem_u8 + (bad_base ? 0u : lut_abs - sbase));
+  float* stage = reinterpret_cast<float*>(smem_u8 + (bad_base ? 0u : hist_abs - sbase));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // warps w, w+4, .. share histogram w % 4: one scheduler serves all turns on it
-  const int hidx = warp % kNHist, role = warp / kNHist;
   const bool lane_live = lane < LB;
-  float* my_p = pbuf + warp * 64;
-  // byte permutes that put an index byte into byte 1 of these give addresses
-  const uint32_t hx = ((1u + static_cast<uint32_t>(hidx >> 1)) << 16) |
-                      static_cast<uint32_t>((hidx & 1) * 128 + lane * 4);
-  uint32_t lx[J];                                      // (value >> 1) = LUT word of lookup s
+  // Byte permutes that put an index byte into byte 1 of these give addresses.
+  // Key lookup s of slot `lane` reads LUT column lane + s (the replicated
+  // columns make the modulo unnecessary): the address of lookup s is
+  // perm(lxb) + 4s. Value update s goes to histogram column (lane + s) % LB.
+  const uint32_t lxb = lut_abs | static_cast<uint32_t>(lane * 4);
+  uint32_t hx[J];
 #pragma unroll
-  for (int s = 0; s < J; ++s) lx[s] = 0x10000u | (8u * static_cast<uint32_t>((lane + s) % LB));
-  // turns on histogram hidx run role 0, 1, .., kPerHist-1, 0, ..
-  const uint32_t bar_wait = smem_addr(mbar + hidx * kPerHist + role);
-  const uint32_t bar_give = smem_addr(mbar + hidx * kPerHist + (role + 1) % kPerHist);
+  for (int s = 0; s < J; ++s) hx[s] = hist_abs | (4u * static_cast<uint32_t>((lane + s) % LB));
   const int bpp = p.Pg / LB;
   const uint32_t bpp_magic = 0xFFFFFFFFu / static_cast<uint32_t>(bpp) + 1u;
 
@@ -470,15 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   int hq = static_cast<int>(off / units_b);
   int pu_start = static_cast<int>(off % units_b);     // unit offset inside the pair
   long long u = u_lo;
-
-  if (!bad_base) {
-    if (tid < kNHist * kPerHist) mbar_init(smem_addr(mbar + tid), 32u);
-    if (tid == 0) flags[0] = 0;
-    __syncthreads();
-    if (role == kPerHist - 1) mbar_arrive(bar_give);   // the first turn is role 0's
-  }
-  uint32_t rnd = 0;                                    // rounds taken (same count in all warps of a histogram)
-  bool wait_failed = false;
+  if (bad_base && tid == 0 && p.status != nullptr) atomicOr(p.status, kStatusSharedBase);
 
   while (u < u_hi && b < p.B) {
     const int seg_units = static_cast<int>(min(static_cast<long long>(units_b - pu_start), u_hi - u));
@@ -502,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
     } else {
       const float* cbk = p.cb_k + hkv * p.cb_stride_head;
       const uint16_t* qp = p.q + (static_cast<size_t>(b) * p.Hq + hq) * d;
-      __syncthreads();                                 // previous segment done with LUT and histograms
+      __syncthreads();                                 // previous segment done with LUT, histogram, q
       // the first chunk of the key slice goes out before anything that waits
       for (int i = tid * 4; i < JC * kE * C; i += kThreads * 4) cp_async16(stage + i, cbk + i);
       const float* cbv = p.cb_v + hkv * p.cb_stride_head;
@@ -513,59 +517,78 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       }
       const float qv = (tid < d) ? bf16_bits_to_float(qp[tid]) * p.scale_log2 : 0.f;
 
-      // ---- index ring prologue ----------------------------------------------
+      // ---- this warp's pages and the index ring --------------------------------
+      // warp w streams the segment's pages pg_lo + w + k*kNW (k = 0, 1, ..), each
+      // as bpp blocks; its t-th block is block t % bpp of its page t / bpp.
+      // Chunk ch holds blocks [ch*KB, (ch+1)*KB) of every warp; its items are
+      // the KB key blocks, then the same KB value blocks.
       const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
       const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages_per_seq;
       auto pages_of = [&](int w) { return (pg_hi > pg_lo + w) ? (pg_hi - pg_lo - w + kNW - 1) / kNW : 0; };
       const int my_first = pg_lo + warp;
       const int n_my_pages = pages_of(warp);
       const int n_blocks = n_my_pages * bpp;
-      // rounds of two blocks; all warps of a histogram take the largest count
-      int most_pages = 0;
-#pragma unroll
-      for (int k = 0; k < kPerHist; ++k) most_pages = max(most_pages, pages_of(hidx + kNHist * k));
-      const int n_rounds = (most_pages * bpp + 1) / 2;
-      int i0 = 0;
+      const int n_chunks = (pages_of(0) * bpp + KB - 1) / KB;   // CTA-uniform (warp 0 has the most)
+      int i0 = 0;                                      // page-table window: pages [i0, i0 + 64)
       auto bt_entry = [&](int i) -> int { return (i < n_my_pages) ? bt[my_first + i * kNW] : -1; };
       int bt_cur = bt_entry(lane);                     // requested now, used after the slice lands
       int bt_nxt = bt_entry(32 + lane);
-      BlockRegs<J> ring[kRing] = {};
+      // L2 prefetch of pages [k0, k1) of this warp's list
+      auto prefetch_pages = [&](int k0, int k1) {
+        k1 = min(k1, n_my_pages);
+        const int a = lane + i0, c = lane + i0 + 32;
+        if (a >= k0 && a < k1 && bt_cur >= 0 && bt_cur < p.n_pages)
+          prefetch_l2_bulk(pool_h + static_cast<int64_t>(bt_cur) * p.page_bytes,
+                           static_cast<uint32_t>(p.page_bytes));
+        if (c >= k0 && c < k1 && bt_nxt >= 0 && bt_nxt < p.n_pages)
+          prefetch_l2_bulk(pool_h + static_cast<int64_t>(bt_nxt) * p.page_bytes,
+                           static_cast<uint32_t>(p.page_bytes));
+      };
+      BlockRegs<J> ring[kRing];
+#pragma unroll
+      for (int k = 0; k < kRing; ++k) ring[k].base = -1;
       // a cleared block keeps whatever bytes it held: every byte value
-      // addresses a valid row, and base = -1 masks its scores and skips it
-      auto clear = [&](BlockRegs<J>& r) { r.base = -1; };
-      auto issue = [&](int k, BlockRegs<J>& r) {
-        if (k >= n_blocks) {                             // warp-uniform
-          clear(r);
+      // addresses a valid row, and base = -1 masks and skips it
+      auto issue = [&](int i, BlockRegs<J>& r) {
+        const int ch = i / (2 * KB);
+        const int pos = i - ch * 2 * KB;
+        const int kv = pos >= KB ? 1 : 0;
+        const int t = ch * KB + (pos - kv * KB);
+        if (pos == 0) {                                  // first item of a chunk (warp-uniform)
+          const int kmin = static_cast<int>(__umulhi(static_cast<uint32_t>(ch * KB), bpp_magic));
+          if (kmin >= i0 + 32) {                         // slide the page-table window
+            bt_cur = bt_nxt;
+            i0 += 32;
+            bt_nxt = bt_entry(i0 + 32 + lane);
+          }
+          const int knext = static_cast<int>(__umulhi(static_cast<uint32_t>((ch + 1) * KB), bpp_magic));
+          prefetch_pages(kmin + kPrefetchPages, knext + kPrefetchPages);
+        }
+        if (t >= n_blocks) {                             // warp-uniform
+          r.base = -1;
           return;
         }
-        const int pi = static_cast<int>(__umulhi(static_cast<uint32_t>(k), bpp_magic));
-        const int blk = k - pi * bpp;
-        if (pi >= i0 + 32) {                             // warp-uniform
-          bt_cur = bt_nxt;
-          i0 += 32;
-          bt_nxt = bt_entry(i0 + 32 + lane);
-        }
-        if (blk == 0) {                                  // first block of a page: prefetch ahead
-          const int tgt = pi + kPrefetchPages;           // tgt - i0 < 64: inside cur or nxt
-          const int src = (tgt - i0 < 32) ? bt_cur : bt_nxt;
-          const int pf = __shfl_sync(0xffffffffu, src, (tgt - i0) & 31);
-          if (lane == 0 && tgt < n_my_pages && pf >= 0 && pf < p.n_pages)
-            prefetch_l2_bulk(pool_h + static_cast<int64_t>(pf) * p.page_bytes,
-                             static_cast<uint32_t>(p.page_bytes));
-        }
-        const int phys = __shfl_sync(0xffffffffu, bt_cur, pi - i0);
+        const int pi = static_cast<int>(__umulhi(static_cast<uint32_t>(t), bpp_magic));
+        const int blk = t - pi * bpp;
+        const int src = (pi - i0 < 32) ? bt_cur : bt_nxt;
+        const int phys = __shfl_sync(0xffffffffu, src, (pi - i0) & 31);
         const int pg = my_first + pi * kNW;
         r.valid = min(p.Pg, n_vq - pg * p.Pg);
         r.base = blk * LB;
-        if (phys < 0 || phys >= p.n_pages || r.base >= r.valid) {   // nothing to read
-          clear(r);
+        if (phys < 0 || phys >= p.n_pages) {             // a page-table entry outside the pool
+          if (lane == 0 && p.status != nullptr) atomicOr(p.status, kStatusBadPage);
+          r.base = -1;
           return;
         }
-        load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, p.Pg, blk,
-                      lane, r);
+        if (r.base >= r.valid) {                         // past the sequence's last token
+          r.base = -1;
+          return;
+        }
+        load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, blk, kv, lane,
+                      r);
       };
 
-      // ---- key LUT from the key slice staged in the histogram windows ----------
+      // ---- key LUT from the key slice staged in the histogram window ----------
       if (tid < d) qs[tid] = qv;
 #pragma unroll 1
       for (int j0 = 0; j0 < J; j0 += JC) {
@@ -577,9 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         cp_async_wait_all();
         __syncthreads();
         if (j0 == 0) {                                 // the page table has landed: first index blocks
-          if (lane < kPrefetchPages && lane < n_my_pages && bt_cur >= 0 && bt_cur < p.n_pages)
-            prefetch_l2_bulk(pool_h + static_cast<int64_t>(bt_cur) * p.page_bytes,
-                             static_cast<uint32_t>(p.page_bytes));
+          prefetch_pages(0, kPrefetchPages);
 #pragma unroll
           for (int k = 0; k < kRing; ++k) issue(k, ring[k]);
         }
@@ -590,158 +611,125 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           const int e = (it / JC) * 32 + lane, jj = (it % JC + lane) % JC, j = j0 + jj;
           const float v = dot_c<C>(qs + j * C, stage + (static_cast<size_t>(jj) * kE + e) * C);
 #pragma unroll
-          for (int r = 0; r < T::R; ++r) lut[e * 32 + j + r * J] = v;
+          for (int c = j; c < 64; c += J) lut[e * 64 + c] = v;   // every column holding group j
         }
       }
       __syncthreads();                                 // LUT complete; staging area free
-      for (uint32_t a = kHistAbs + 16u * tid; a < kHistEnd; a += 16u * kThreads)
-        asm volatile("st.shared.v4.f32 [%0], {%1, %1, %1, %1};" ::"r"(a), "f"(0.f) : "memory");
-      if (tid < kNHist) hm[tid] = -INFINITY;
-      __syncthreads();                                 // histograms zero, maxima reset
+      for (uint32_t a = hist_abs + 16u * tid; a < hist_abs + kHistBytes; a += 16u * kThreads)
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+      __syncthreads();                                 // histogram zero
 
       // ---- stream -------------------------------------------------------------
-      float m_seen = -INFINITY;                        // pair maximum this warp's l refers to
-      float l_lane = 0.f;
       auto key_scores = [&](const BlockRegs<J>& r) -> float {
+        if (r.base < 0) return -INFINITY;              // warp-uniform
         float xa[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t ad[J];
 #pragma unroll
-        for (int s = 0; s < J; ++s)
-          xa[s & 3] += lds_lut(__byte_perm(r.k[s >> 2], lx[s], 0x7604u | (uint32_t(s & 3) << 4)) >> 1);
-        const bool valid = r.base >= 0 && lane_live && (r.base + lane) < r.valid;
+        for (int s = 0; s < J; ++s) ad[s] = __byte_perm(r.w[s >> 2], lxb, 0x7604u | (uint32_t(s & 3) << 4));
+        constexpr_for<J>([&](auto S) { xa[S.value & 3] += lds_lut<4 * S.value>(ad[S.value]); });
+        const bool valid = lane_live && (r.base + lane) < r.valid;
         return valid ? (xa[0] + xa[1]) + (xa[2] + xa[3]) : -INFINITY;
       };
-      auto value_pass = [&](const BlockRegs<J>& r, const float* pp) {
+      // histogram updates of one value block, lane = slot: the slot's weight
+      // w = rn(2^(x - m) * 2^kFixBits) goes to row idx_V[slot][j] of column
+      // (lane + s) % LB for each byte s of its rotated row; carries out of a low
+      // word go to its high word
+      auto value_pass = [&](const BlockRegs<J>& r, float x, float m) {
         if (r.base < 0) return;                        // warp-uniform
         if constexpr (LB < 32) {
           if (!lane_live) return;
         }
-        pp += (lane / J) * J;
-        float4 p4 = *reinterpret_cast<const float4*>(pp);
+        uint32_t w = __float2uint_rn(fast_exp2(x - m) * kFixScale);   // 0 for x = -inf
+        w = min(w, 1u << kFixBits);
+        const uint32_t nw = ~w;
+        uint32_t a[4], o[4];
 #pragma unroll
-        for (int i = 0; i < J; i += 4) {
-          const uint32_t w = r.v[i >> 2];
-          const uint32_t a0 = __byte_perm(w, hx, 0x7604u), a1 = __byte_perm(w, hx, 0x7614u);
-          const uint32_t a2 = __byte_perm(w, hx, 0x7624u), a3 = __byte_perm(w, hx, 0x7634u);
-          // fold each weight into the last slot of the four with the same row
-          float q1 = p4.y, q2 = p4.z, q3 = p4.w;
-          if (a1 == a0) q1 += p4.x;
-          if (a2 == a0) q2 += p4.x;
-          if (a2 == a1) q2 += p4.y;
-          if (a3 == a0) q3 += p4.x;
-          if (a3 == a1) q3 += p4.y;
-          if (a3 == a2) q3 += p4.z;
-          const float o0 = lds_h(a0), o1 = lds_h(a1), o2 = lds_h(a2), o3 = lds_h(a3);
-          // the next batch's weights (never written during the pass) before this batch's stores
-          const float4 p4n = (i + 4 < J) ? *reinterpret_cast<const float4*>(pp + i + 4) : p4;
-          sts_h(a0, o0 + p4.x);
-          sts_h(a1, o1 + q1);
-          sts_h(a2, o2 + q2);
-          sts_h(a3, o3 + q3);
-          p4 = p4n;
+        for (int i = 0; i < J / 4; ++i) {
+          uint32_t an[4], on[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) an[k] = __byte_perm(r.w[i], hx[4 * i + k], 0x7604u | (uint32_t(k) << 4));
+          hist_add4(an, w, on);
+          if (i > 0) hist_carry4(a, o, nw);            // the previous four, whose old words are back
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            a[k] = an[k];
+            o[k] = on[k];
+          }
+        }
+        hist_carry4(a, o, nw);
+      };
+      // exact rescale of the 64-bit cells by 2^-sh when the reference maximum rises
+      auto rescale = [&](int sh) {
+        for (int cell = tid; cell < kE * 32; cell += kThreads) {
+          const uint32_t ad = hist_abs + (static_cast<uint32_t>(cell >> 5) << 8) +
+                              (static_cast<uint32_t>(cell & 31) << 2);
+          uint32_t lo = lds_u32(ad), hi = lds_u32(ad + 128u);
+          if (sh >= 64) {
+            lo = 0u;
+            hi = 0u;
+          } else if (sh >= 32) {
+            lo = hi >> (sh - 32);
+            hi = 0u;
+          } else {
+            lo = __funnelshift_r(lo, hi, sh);
+            hi >>= sh;
+          }
+          sts_u32(ad, lo);
+          sts_u32(ad + 128u, hi);
         }
       };
-      // One round: key scores and (against the maximum this warp saw last)
-      // weights outside the turn, the histogram updates inside.
-      auto round = [&](const BlockRegs<J>& ra, const BlockRegs<J>& rb) {
-        const float xa = key_scores(ra);
-        const float xb = key_scores(rb);
-        const float xl = fmaxf(xa, xb);
-        const bool spec = m_seen != -INFINITY &&
-                          __all_sync(0xffffffffu, !(xl > m_seen + kRescaleSlack));
-        float pa = 0.f, pb = 0.f;
-        if (spec) {                                    // warp-uniform
-          pa = fast_exp2(xa - m_seen);
-          pb = fast_exp2(xb - m_seen);
-          my_p[lane] = pa;
-          my_p[32 + lane] = pb;
-        }
-        if (!wait_failed && !mbar_wait(bar_wait, rnd & 1u)) wait_failed = true;
-        ++rnd;
-        float m = hm[hidx];
-        const bool keep = spec && m == m_seen;         // warp-uniform
-        if (m != m_seen) {                             // another warp raised the maximum
-          if (m_seen != -INFINITY) l_lane *= fast_exp2(m_seen - m);
-          m_seen = m;
-        }
-        if (!keep && __any_sync(0xffffffffu, xl > m + kRescaleSlack)) {   // warp-uniform, rare
-          const float xm = warp_max(xl);
-          if (m != -INFINITY) {
-            const float f = fast_exp2(m - xm);
-            if (lane_live) {
-              for (int e = 0; e < kE; ++e) {
-                const uint32_t a = hx | (static_cast<uint32_t>(e) << 8);
-                sts_h(a, lds_h(a) * f);
-              }
-            }
-            l_lane *= f;
-          }
-          m = xm;
-          m_seen = xm;
-          if (lane == 0) hm[hidx] = xm;
-        }
-        if (m != -INFINITY) {                          // warp-uniform
-          if (!keep) {
-            pa = fast_exp2(xa - m);                    // 0 for xa = -inf
-            pb = fast_exp2(xb - m);
-            my_p[lane] = pa;
-            my_p[32 + lane] = pb;
-          }
-          l_lane += pa + pb;
-          __syncwarp();
-          value_pass(ra, my_p);
-          value_pass(rb, my_p + 32);
-          __syncwarp();                                // my_p is rewritten next round
-        }
-        mbar_arrive(bar_give);                         // all lanes: releases this turn's writes
-      };
 
-      for (int r0 = 0; r0 < n_rounds; r0 += kRing / 2) {
+      float m_cur = -INFINITY;                         // integer reference maximum (CTA-uniform)
+#pragma unroll 1
+      for (int ch = 0; ch < n_chunks; ++ch) {
+        const int ib = ch * 2 * KB;
+        float xs[KB];
+        float cm = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < kRing / 2; ++h) {
-          if (r0 + h < n_rounds) {                     // warp-uniform
-            round(ring[2 * h], ring[2 * h + 1]);
-            issue(2 * (r0 + h) + kRing, ring[2 * h]);
-            issue(2 * (r0 + h) + kRing + 1, ring[2 * h + 1]);
+        for (int q = 0; q < KB; ++q) {                 // key phase
+          xs[q] = key_scores(ring[q % kRing]);
+          cm = fmaxf(cm, xs[q]);
+          issue(ib + q + kRing, ring[q % kRing]);
+        }
+        cm = warp_max(cm);
+        if (lane == 0) wmax[(ch & 1) * kNW + warp] = cm;
+        __syncthreads();                               // every warp's chunk maximum
+        float cmax = (lane < kNW) ? wmax[(ch & 1) * kNW + lane] : -INFINITY;
+        cmax = warp_max(cmax);
+        if (cmax != -INFINITY) {                       // CTA-uniform
+          const float m_new = fmaxf(m_cur, ceilf(cmax));
+          if (m_cur != -INFINITY && m_new > m_cur) {   // earlier chunks' weights shrink by 2^-(m_new - m_cur)
+            rescale(static_cast<int>(fminf(m_new - m_cur, 64.f)));
+            __syncthreads();
           }
+          m_cur = m_new;
+        }
+#pragma unroll
+        for (int q = 0; q < KB; ++q) {                 // value phase
+          if (m_cur != -INFINITY) value_pass(ring[(KB + q) % kRing], xs[q], m_cur);   // CTA-uniform
+          issue(ib + KB + q + kRing, ring[(KB + q) % kRing]);
         }
       }
-      const float l_w = warp_sum(l_lane);
-      if (lane == 0) {
-        wstat[warp] = m_seen;
-        wstat[kNW + warp] = l_w;
-        if (wait_failed) atomicOr(flags, 1);
-      }
-      __syncthreads();
+      __syncthreads();                                 // every update landed
 
-      // ---- merge the histograms, contract with the value slice -------------------
-      float Mh = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < kNHist; ++h) Mh = fmaxf(Mh, hm[h]);
-      if (Mh == -INFINITY) {                           // nothing valid: an empty record
+      // ---- histogram to float, contraction with the value slice ---------------
+      if (m_cur == -INFINITY) {                        // nothing valid: an empty record
         if (tid == 0) {
-          rec[0] = (flags[0] != 0) ? NAN : -INFINITY;
+          rec[0] = -INFINITY;
           rec[1] = 0.f;
         }
       } else {
-        float L = 0.f;
-#pragma unroll
-        for (int w = 0; w < kNW; ++w)
-          if (wstat[w] != -INFINITY) L += wstat[kNW + w] * fast_exp2(wstat[w] - Mh);
-        float fh[kNHist];
-#pragma unroll
-        for (int h = 0; h < kNHist; ++h) fh[h] = (hm[h] == -INFINITY) ? 0.f : fast_exp2(hm[h] - Mh);
         // W[e][j]: lane = column, rows warp + kNW*k; replicas of a group are summed
-        constexpr int NR = (kE + kNW - 1) / kNW;       // rows per warp
-        const float* hist = stage;                     // the histogram windows as floats
+        constexpr int NR = kE / kNW;                   // rows per warp
         float wv[NR];
 #pragma unroll
         for (int k = 0; k < NR; ++k) {
           const int e = warp + kNW * k;
           float v = 0.f;
-          if (e < kE && lane_live) {
-#pragma unroll
-            for (int h = 0; h < kNHist; ++h)
-              v = fmaf(fh[h], hist[(h >> 1) * 16384 + e * 64 + (h & 1) * 32 + lane], v);
+          if (lane_live) {
+            const uint32_t ad = hist_abs + (static_cast<uint32_t>(e) << 8) + 4u * lane;
+            const uint32_t lo = lds_u32(ad), hi = lds_u32(ad + 128u);
+            v = (__uint2float_rn(hi) * 4294967296.0f + __uint2float_rn(lo)) * kFixInv;
           }
 #pragma unroll
           for (int o = (T::R / 2) * J; o >= J; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
@@ -753,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
 #pragma unroll
         for (int k = 0; k < NR; ++k) {
           const int e = warp + kNW * k;
-          if (e < kE && lane < J) wt[lane * EP + e] = wv[k];
+          if (lane < J) wt[lane * EP + e] = wv[k];
         }
         __syncthreads();
         // o[j*C + ch] = sum_e W[e][j] C_V[j][e][ch]: warp -> groups, lane -> rows lane + 32 i
@@ -781,9 +769,15 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
             if (lane == ch) rec[4 + j * C + ch] = t;
           }
         }
-        if (tid == 0) {
-          rec[0] = (flags[0] != 0) ? NAN : Mh;         // a turn that timed out poisons the pair
-          rec[1] = L;
+        if (warp == kNW - 1) {                         // l = sum_e W[e][j], the same for every group j
+          float l = 0.f;
+#pragma unroll
+          for (int i = 0; i < kE / 32; ++i) l += wt[lane + 32 * i];
+          l = warp_sum(l);
+          if (lane == 0) {
+            rec[0] = m_cur;
+            rec[1] = l;
+          }
         }
       }
     }
@@ -950,7 +944,8 @@ loopvq_status launch_decode(const DecodeArgs& a) {
   p.seq_lens = a.seq_lens;
   p.win_k = static_cast<const uint16_t*>(a.win_k);
   p.win_v = static_cast<const uint16_t*>(a.win_v);
-  p.records = static_cast<float*>(a.workspace);
+  p.status = static_cast<int*>(a.workspace);
+  p.records = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + kStatusBytes);
   p.out = a.out;
   p.lse = a.lse;
   p.B = a.batch;

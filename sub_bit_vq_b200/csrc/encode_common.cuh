@@ -38,16 +38,12 @@ __device__ __forceinline__ void store_index(const EncodeParams& p, int64_t slot,
   }
   const int64_t page = slot / p.Pg;
   const int sl = static_cast<int>(slot % p.Pg);
-  int64_t off;
-  if (p.kv == 0) {                          // K plane: rotated slot rows
-    const int blk = sl / p.LB, rot = sl % p.LB;
-    int pos = j - rot % p.J;
-    if (pos < 0) pos += p.J;
-    off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR + rot * p.GR +
-          pos % p.GR;
-  } else {                                  // V plane: group-major
-    off = static_cast<int64_t>(j) * p.Pg + sl;
-  }
+  // both planes: rotated slot rows in granules
+  const int blk = sl / p.LB, rot = sl % p.LB;
+  int pos = j - rot % p.J;
+  if (pos < 0) pos += p.J;
+  const int64_t off = static_cast<int64_t>(blk) * p.LB * p.J + (pos / p.GR) * p.LB * p.GR +
+                      rot * p.GR + pos % p.GR;
   p.pool[h * p.pool_stride_head + page * p.page_bytes + p.kv * p.plane_bytes + off] =
       static_cast<uint8_t>(e);
 }

@@ -28,6 +28,10 @@ int max_decode_splits(int pairs, int pages);
 // segment records of 4 + d floats.
 constexpr int kMaxStreamCtas = 256;
 
+// Bytes at the start of the decode workspace that hold the status word (an
+// int32 of flag bits); the segment records follow.
+constexpr size_t kStatusBytes = 256;
+
 // Number of multiprocessors of the current device (cached per device).
 // Returns 0 and sets *err when the runtime fails.
 int current_sm_count(loopvq_status* err);

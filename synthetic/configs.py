@@ -85,11 +85,12 @@ SHAPES: dict[str, Shape] = {
     # 0.25 bit, deep recurrence: d=96, 40 kv-heads, 16 loops in groups of 4,
     # c=8 (32-element sub-vectors), batch 32, context 16384, AR(1) loops.
     # The layer count is not given; 4 layers are enough to rotate buffers
-    # past the L2 cache.
+    # past the L2 cache. Pages hold 96 tokens: a multiple of the 24-slot
+    # rotation block of J = 12 groups (and of 16).
     "deep025": Shape("deep025", n_layers=4, n_kv_heads=40, n_q_heads=40,
                      head_dim=96, n_loops=16, loop_group=4, chan_group=8,
                      batch=32, context=16384, kind="ar1", loop_corr=0.8,
-                     seed=1004),
+                     page_tokens=96, seed=1004),
     # Encoder + batch sweep: 16 heads, d=128, 4 loops, g=4, c=4; the encode
     # leg is a 32768-token prefill, the sweep is batch 1..256 at 16384.
     "sweep": Shape("sweep", n_layers=1, n_kv_heads=16, n_q_heads=16,

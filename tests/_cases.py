@@ -162,3 +162,77 @@ def check_indices(gpu_idx: np.ndarray, dist: np.ndarray, rel: float = 1e-5) -> i
     chosen = flat_d[np.arange(flat_d.shape[0]), flat_i]
     assert np.all(chosen - d1 <= rel * d1 + 0.0), "near-tie choice outside the margin"
     return int(((flat_i != ref) & tie).sum())
+
+
+class DeviceDecodeCase:
+    """Decode inputs at full configuration size for one (layer, loop step).
+
+    The pool lives on the GPU only: either random bytes drawn there (seeded),
+    or a pool the caller filled (e.g. with the GPU encoder). The oracle of a
+    pair reads back just that pair's pages. Codebooks, queries and windows
+    are host tensors copied to the GPU once."""
+
+    def __init__(self, shape: Shape, seq_lens, *, loop_step=0, seed=0, q_scale=1.0, cb=None,
+                 pool=None, bt=None, dev="cuda"):
+        self.shape = shape
+        self.seq_lens = list(seq_lens)
+        self.B = len(self.seq_lens)
+        self.layer, self.n_layers, self.t = 0, 1, loop_step
+        self.gamma, self.tau = loop_step // shape.loop_group, loop_step % shape.loop_group
+        H, J, Pg = shape.n_kv_heads, shape.J, shape.page_tokens
+        if bt is None:
+            bt = block_tables(shape, self.B, self.seq_lens, spare_pages=1)
+        self.bt, self.n_pages = bt[0].cpu(), bt[1]
+        self.max_pages = self.bt.shape[1]
+        self.cb = random_codebooks(shape, 1, seed + 7) if cb is None else cb.cpu()
+        if pool is None:
+            g = torch.Generator(device=dev)
+            g.manual_seed(seed)
+            pool = torch.randint(0, 256, (1, H, shape.G, self.n_pages, 2, Pg * J), generator=g,
+                                 dtype=torch.uint8, device=dev)
+        self.pool = pool
+        self.q = (queries(shape, 0, loop_step, batch=self.B).float() * q_scale).to(torch.bfloat16)
+        self.win_k = window_kv(shape, 0, loop_step, 0, batch=self.B)
+        self.win_v = window_kv(shape, 0, loop_step, 1, batch=self.B)
+        self.max_seq_len = max(self.seq_lens + [0])
+        self.sm_scale = 1.0 / math.sqrt(shape.head_dim)
+        self.dev = dev
+
+    config = DecodeCase.config
+    oracle = DecodeCase.oracle
+
+    def indices(self, b: int, hkv: int):
+        s = self.shape
+        n = O.n_vq_tokens(self.seq_lens[b], s.prefix, s.recent)
+        pages = -(-n // s.page_tokens)
+        phys = self.bt[b, :pages].long().to(self.dev)
+        plane = self.pool.view(1, s.n_kv_heads, s.G, self.n_pages, 2, -1)[0, hkv, self.gamma][phys]
+        plane = plane.cpu().numpy()                    # this pair's pages, in table order
+        row = np.arange(pages)
+        return (O.unpack_sequence(plane, n, s.J, row, s.page_tokens, 0),
+                O.unpack_sequence(plane, n, s.J, row, s.page_tokens, 1))
+
+    def run_gpu(self, out_dtype=torch.float32):
+        dev = self.dev
+        cfg = self.config()
+        s = self.shape
+        cb, bt = self.cb.to(dev), self.bt.to(dev)
+        sl = torch.tensor(self.seq_lens, dtype=torch.int32, device=dev)
+        q, wk, wv = self.q.to(dev), self.win_k.to(dev), self.win_v.to(dev)
+        out = torch.full((self.B, s.n_q_heads, s.head_dim), float("nan"), dtype=out_dtype, device=dev)
+        lse = torch.full((self.B, s.n_q_heads), float("nan"), dtype=torch.float32, device=dev)
+        nbytes = L.loopvq_decode_workspace_bytes(cfg, self.B, self.max_seq_len)
+        ws = torch.full((max(nbytes // 4, 1),), float("nan"), dtype=torch.float32, device=dev)
+        L.loopvq_decode_attn(cfg, self.layer, self.t, q, self.pool, cb, bt, sl, wk, wv, out, ws,
+                             self.max_seq_len, lse=lse, sm_scale=self.sm_scale)
+        torch.cuda.synchronize()
+        return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def sample_pairs(B: int, Hq: int, n: int, seed: int, whole=()):
+    """``n`` random (sequence, head) pairs plus every head of the sequences in
+    ``whole``."""
+    r = np.random.default_rng(seed)
+    pairs = {(int(b), int(h)) for b, h in zip(r.integers(0, B, n), r.integers(0, Hq, n))}
+    pairs |= {(b, h) for b in whole for h in range(Hq)}
+    return sorted(pairs)

@@ -170,11 +170,11 @@ def test_kmeans_step_rejects_before_launch():
 
 def test_workspace_bytes_formula():
     cfg = _cfg()
-    # one record (m, l, 2 spare, value histogram [256][J]) of float32 per
-    # (sequence, query head, split)
+    # a 256-byte status area, then one record (m, l, 2 spare, o[d]) of float32
+    # per (pair, streaming CTA) slot: pairs + 256 slots
     n = L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64)
     rec = 4 * (4 + cfg.head_dim)
-    assert n % rec == 0 and n >= rec * 2 * cfg.n_q_heads
+    assert n == 256 + rec * (2 * cfg.n_q_heads + 256)
     # more sequences need more records
     assert L.loopvq_decode_workspace_bytes(cfg, 4, 72 + 5 * 64) > n
     assert L.loopvq_decode_workspace_bytes(cfg, 0, 10) == 0
@@ -190,9 +190,18 @@ def test_python_api_exports_the_documented_calls():
     for name in ("LoopVQConfig", "loopvq_cache_layout", "loopvq_encode", "loopvq_kmeans_assign_bytes",
                  "loopvq_kmeans_step", "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
                  "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn",
-                 "loopvq_status_string"):
+                 "loopvq_decode_attn_noalloc", "loopvq_status_string"):
         assert callable(getattr(L, name)), name
     cfg = _cfg()
     lay = L.loopvq_cache_layout(cfg)
     assert lay["bits_per_element"] == 0.5
     assert L.loopvq_kmeans_assign_bytes(cfg, 7) == 3 * 32 * 7
+
+
+def test_static_scratch_size_matches_the_header():
+    # the binding's copy of LOOPVQ_STATIC_SCRATCH_BYTES is the header's value
+    text = open(os.path.join(ROOT, "include", "loopvq.h")).read()
+    m = re.search(r"#define\s+LOOPVQ_STATIC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
+    assert m, "LOOPVQ_STATIC_SCRATCH_BYTES not found in include/loopvq.h"
+    assert int(m.group(1)) << int(m.group(2)) == B.LOOPVQ_STATIC_SCRATCH_BYTES
+    assert L.LOOPVQ_STATIC_SCRATCH_BYTES == B.LOOPVQ_STATIC_SCRATCH_BYTES

@@ -344,9 +344,12 @@ def test_plane_offsets_hand_worked():
     assert O.plane_offset(31, 7, 12) == 288 + 28
     # J=24, granule 8. slot 5, group 6 -> pos 1 -> 5*8 + 1.
     assert O.plane_offset(5, 6, 24) == 41
-    # V plane is group-major: slot 5, group 3 with 64-slot pages -> 3*64 + 5.
-    assert O.plane_offset(5, 3, 32, 1, 64) == 197
-    assert O.plane_offset(95, 11, 12, 1, 96) == 11 * 96 + 95
+    # The V plane has the same layout. J=32: slot 5, group 3 -> pos 30 ->
+    # granule 1 (512), row 5 (80), byte 14.
+    assert O.plane_offset(5, 3, 32, 1, 64) == 512 + 80 + 14
+    # J=12: slot 95 is row 23 of block 3 (3*288 = 864): group 11 -> pos 0 ->
+    # granule 0, row 23 (92), byte 0.
+    assert O.plane_offset(95, 11, 12, 1, 96) == 864 + 92
 
 
 def test_pack_unpack_round_trip():
@@ -509,3 +512,36 @@ def test_lloyd_step_shared_weights_equal_repeated_per_token_weights():
     i2, n2 = O.kmeans_step_group_ref(X, cb, np.repeat(shared, X.shape[1], axis=1))
     np.testing.assert_array_equal(i1, i2)
     np.testing.assert_allclose(n1, n2, rtol=0, atol=0)
+
+
+def test_weighted_distortion_hand_worked():
+    # g = 2 loop steps, c = 2 channels, one head, d = 2 (J = 1), D = 4; two
+    # tokens, two centroids, unequal weights. Loop-major sub-vectors:
+    #   s0 = (1, 2, 3, 4), s1 = (0, -1, 2, 0); codewords c0 = (1, 1, 1, 1),
+    #   c1 = (0, 0, 2, 2); weights w0 = (2, 1, 0.5, 3), w1 = (1, 4, 2, 0).
+    # Assignment (0, 1):
+    #   token 0: w0 . (0, 1, 2, 3)^2 = 0 + 1 + 2 + 27 = 30
+    #   token 1: w1 . (0, -1, 0, -2)^2 = 0 + 4 + 0 + 0 = 4           -> 34
+    # Unweighted: 14 + 5 = 19. Assignment (1, 0):
+    #   w0 . (1, 2, 1, 2)^2 = 18.5;  w1 . (-1, -2, 1, -1)^2 = 19     -> 37.5
+    # Weights shared over tokens (token 0's vector for both):
+    #   30 + (2, 1, 0.5, 3) . (0, 1, 0, 4) = 30 + 13                   -> 43
+    X = np.zeros((2, 2, 1, 2))
+    X[0, 0, 0], X[1, 0, 0] = (1, 2), (3, 4)
+    X[0, 1, 0], X[1, 1, 0] = (0, -1), (2, 0)
+    cb = np.zeros((1, 2, 1, 2, 2))                      # [H][g][J][E][c]
+    cb[0, 0, 0, 0], cb[0, 1, 0, 0] = (1, 1), (1, 1)
+    cb[0, 0, 0, 1], cb[0, 1, 0, 1] = (0, 0), (2, 2)
+    w = np.zeros((2, 2, 1, 2))
+    w[0, 0, 0], w[1, 0, 0] = (2, 1), (0.5, 3)
+    w[0, 1, 0], w[1, 1, 0] = (1, 4), (2, 0)
+    a01 = np.array([[[0]], [[1]]], dtype=np.uint8)        # [N][H][J]
+    a10 = np.array([[[1]], [[0]]], dtype=np.uint8)
+    assert O.weighted_distortion_ref(X, cb, a01, w) == 34.0
+    assert O.weighted_distortion_ref(X, cb, a01, None) == 19.0
+    assert O.weighted_distortion_ref(X, cb, a10, w) == 37.5
+    assert O.weighted_distortion_ref(X, cb, a01, w[:, :1]) == 43.0
+    # the encoder agrees: under these weights token 0 prefers c1 (18.5 < 30)
+    idx, dist = O.encode_group_ref(X, cb, w)
+    assert dist[0, 0, 0].tolist() == [30.0, 18.5] and dist[1, 0, 0].tolist() == [19.0, 4.0]
+    assert idx[:, 0, 0].tolist() == [1, 1]

@@ -38,30 +38,60 @@ def _inputs(case, dev="cuda"):
         lse=torch.full((case.B, s.n_q_heads), float("nan"), device=dev))
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
-    case = DecodeCase(SHAPE, [60, 73, 900, 3000], layer=1, n_layers=2, loop_step=2, seed=5)
-    a = _inputs(case)
+def _workspace_reference(case, a):
+    """out/lse of the workspace entry point, its scratch filled with NaN."""
     need = L.loopvq_decode_workspace_bytes(a["cfg"], case.B, case.max_seq_len)
     assert 0 < need <= B.LOOPVQ_STATIC_SCRATCH_BYTES
-    ws = torch.empty(need // 4 + 1, device="cuda")
+    ws = torch.full((need // 4 + 1,), float("nan"), device="cuda")
     L.loopvq_decode_attn(a["cfg"], case.layer, case.t, a["q"], a["pool"], a["cb"], a["bt"], a["sl"],
                          a["wk"], a["wv"], a["out"], ws, case.max_seq_len, lse=a["lse"],
                          sm_scale=case.sm_scale)
     torch.cuda.synchronize()
-    ref_out, ref_lse = a["out"].cpu().numpy(), a["lse"].cpu().numpy()
+    return a["out"].cpu().numpy(), a["lse"].cpu().numpy()
+
+
+def _noalloc(case, a):
+    out = torch.full_like(a["out"], float("nan"))
+    lse = torch.full_like(a["lse"], float("nan"))
+    B.loopvq_decode_attn_noalloc(a["cfg"], case.layer, case.t, a["q"], a["pool"], a["cb"],
+                                 a["bt"], a["sl"], a["wk"], a["wv"], out, case.max_seq_len,
+                                 lse=lse, sm_scale=case.sm_scale)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+def _compare(case, got, ref):
+    (o, ls), (ro, rl) = got, ref
+    for b in range(case.B):
+        for h in range(case.shape.n_q_heads):
+            if case.seq_lens[b] == 0:
+                assert np.all(o[b, h] == 0) and ls[b, h] == -np.inf
+                continue
+            rel = np.max(np.abs(o[b, h] - ro[b, h])) / np.max(np.abs(ro[b, h]))
+            assert rel <= TOL_F32_REL, (b, h, rel)
+            assert abs(ls[b, h] - rl[b, h]) <= TOL_LSE
+
+
+def test_noalloc_matches_workspace_entry_point_on_two_calls():
+    # Two different calls in a row: a batch with one long sequence, then a
+    # smaller batch of short sequences. The second call writes fewer split
+    # records than the first left in the shared static array, so a record it
+    # did not write would surface as a mismatch.
+    first = DecodeCase(SHAPE, [60, 73, 900, 20000], layer=1, n_layers=2, loop_step=2, seed=5)
+    second = DecodeCase(SHAPE.with_(batch=3), [75, 0, 640], layer=0, n_layers=2, loop_step=1,
+                        seed=6)
+    for case in (first, second):
+        a = _inputs(case)
+        ref = _workspace_reference(case, a)
+        _compare(case, _noalloc(case, a), ref)
+
+
+def test_noalloc_repeated_call_gives_the_same_result():
+    case = DecodeCase(SHAPE, [200, 1500, 73, 4000], layer=0, n_layers=2, loop_step=3, seed=7)
+    a = _inputs(case)
+    ref = _workspace_reference(case, a)
     for _ in range(2):
-        out = torch.full_like(a["out"], float("nan"))
-        lse = torch.full_like(a["lse"], float("nan"))
-        B.loopvq_decode_attn_noalloc(a["cfg"], case.layer, case.t, a["q"], a["pool"], a["cb"],
-                                     a["bt"], a["sl"], a["wk"], a["wv"], out, case.max_seq_len,
-                                     lse=lse, sm_scale=case.sm_scale)
-        torch.cuda.synchronize()
-        o, ls = out.cpu().numpy(), lse.cpu().numpy()
-        for b in range(case.B):
-            for h in range(SHAPE.n_q_heads):
-                rel = np.max(np.abs(o[b, h] - ref_out[b, h])) / np.max(np.abs(ref_out[b, h]))
-                assert rel <= TOL_F32_REL, (b, h, rel)
-                assert abs(ls[b, h] - ref_lse[b, h]) <= TOL_LSE
+        _compare(case, _noalloc(case, a), ref)
 
 
 def test_noalloc_rejects_sizes_beyond_the_static_scratch():
