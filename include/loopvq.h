@@ -52,12 +52,26 @@ typedef enum {
 
 enum { LOOPVQ_DTYPE_BF16 = 0, LOOPVQ_DTYPE_F32 = 1 };
 
+/* Flag bits of a decode call's status word (the first int32 of its
+ * workspace), set by the kernels, never cleared by them. */
+enum {
+  /* a block_table entry of a page the call reads lies outside [0, n_pages);
+   * the page was skipped */
+  LOOPVQ_DECODE_STATUS_BAD_PAGE = 1,
+  /* the streaming kernel's shared-memory allocation did not start where its
+   * address arithmetic needs it; its records are NaN (the host checks this
+   * before launching and returns LOOPVQ_ERR_UNSUPPORTED, so this bit means a
+   * device that changed under the library) */
+  LOOPVQ_DECODE_STATUS_SHARED_BASE = 2
+};
+
 /*
  * Static shape of one LoopVQ cache. Supported: head_dim % 8 == 0 and
  * head_dim <= 256; chan_group in {1,2,4,8,16} dividing head_dim; J = d/c a
  * multiple of 4 and at most 32; n_loops % loop_group == 0; D = c*g <= 32;
- * n_centroids == 256; page_tokens a multiple of the rotation block
- * LB = floor(32/J)*J and of 16, at most 256; n_q_heads % n_kv_heads == 0.
+ * n_centroids == 256; page_tokens a multiple of 16, at most 256, and a
+ * power-of-two multiple (1, 2, 4, ..) of the rotation block LB =
+ * floor(32/J)*J; n_q_heads % n_kv_heads == 0.
  */
 typedef struct {
   uint32_t struct_size;      /* sizeof(loopvq_config) */
@@ -214,9 +228,10 @@ loopvq_status loopvq_kmeans_step(const loopvq_config* cfg, int layer, int loop_g
 
 /*
  * Bytes of scratch that loopvq_decode_attn needs for `batch` sequences of
- * at most `max_seq_len` tokens: (batch*Hq + 256) segment records of
- * 4 + head_dim float32 (a segment's softmax maximum and sum and its
- * unnormalised output). Host only, pure.
+ * at most `max_seq_len` tokens: a 256-byte status area (below), then
+ * (batch*Hq + 256) segment records of 4 + head_dim float32 (a segment's
+ * softmax maximum and sum and its unnormalised output), then batch*Hq key
+ * lookup tables of 256 x J float32. Host only, pure.
  */
 size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int max_seq_len);
 
@@ -246,7 +261,12 @@ size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int ma
  *               out = 0 and lse = -inf.
  *  workspace    device scratch of at least
  *               loopvq_decode_workspace_bytes(cfg, batch, max_seq_len),
- *               16-byte aligned; its contents need no initialisation.
+ *               16-byte aligned. Its contents need no initialisation except
+ *               the status word, the int32 at byte 0: the kernels OR
+ *               LOOPVQ_DECODE_STATUS_* bits into it and never clear it. A
+ *               caller that wants to know zeroes it before the call and
+ *               reads it after synchronising; a nonzero word means the
+ *               outputs of that call are not to be trusted.
  */
 loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_step, int batch,
                                  int max_seq_len, const void* q, const uint8_t* pool,
@@ -284,7 +304,7 @@ loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_s
  * kernels overlap on the GPU, e.g. on two streams without ordering, race
  * on it and give undefined results.
  */
-#define LOOPVQ_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+#define LOOPVQ_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 loopvq_status loopvq_decode_attn_noalloc(const loopvq_config* cfg, int layer, int loop_step,
                                          int batch, int max_seq_len, const void* q,
                                          const uint8_t* pool, const float* codebooks,

@@ -250,7 +250,7 @@ def loopvq_decode_attn(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.T
     _check("loopvq_decode_attn", st)
 
 
-LOOPVQ_STATIC_SCRATCH_BYTES = 4 << 20
+LOOPVQ_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 def loopvq_decode_attn_noalloc(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.Tensor,

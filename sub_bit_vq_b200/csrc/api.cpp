@@ -70,6 +70,7 @@ loopvq_status make_geometry(const loopvq_config* cfg, Geometry* geo) {
   g.GR = (g.J % 16 == 0) ? 16 : (g.J % 8 == 0) ? 8 : 4;
   g.LB = (32 / g.J) * g.J;
   if (g.Pg % g.LB != 0 || g.Pg % 16 != 0 || g.Pg > 256) return LOOPVQ_ERR_UNSUPPORTED;
+  if (((g.Pg / g.LB) & (g.Pg / g.LB - 1)) != 0) return LOOPVQ_ERR_UNSUPPORTED;   // blocks per page: 2^k
   g.plane_bytes = static_cast<int64_t>(g.Pg) * g.J;
   g.page_bytes = 2 * g.plane_bytes;
   if (!mul_ok(g.page_bytes, g.n_pages, &g.pool_stride_group)) return LOOPVQ_ERR_INVALID_ARG;
@@ -167,11 +168,12 @@ loopvq_status loopvq_cache_layout(const loopvq_config* cfg, loopvq_layout* out) 
 size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int max_seq_len) {
   Geometry g;
   if (loopvq::make_geometry(cfg, &g) != LOOPVQ_OK || batch <= 0 || max_seq_len < 0) return 0;
-  // one record (m, l, two spare floats, unnormalised output o[d]) per
-  // (pair, streaming CTA) segment: record slots pair + cta never collide, so
-  // pairs + CTAs slots suffice
+  // the status word; one record (m, l, two spare floats, unnormalised output
+  // o[d]) per (pair, streaming CTA) segment: record slots pair + cta never
+  // collide, so pairs + CTAs slots suffice; one key lookup table per pair
   const size_t slots = static_cast<size_t>(batch) * g.Hq + loopvq::kMaxStreamCtas;
-  return loopvq::kStatusBytes + slots * (4 + static_cast<size_t>(g.d)) * sizeof(float);
+  return loopvq::kStatusBytes + slots * (4 + static_cast<size_t>(g.d)) * sizeof(float) +
+         loopvq::decode_lut_bytes(batch * g.Hq, g.J);
 }
 
 loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_idx, int kv,

@@ -1,47 +1,52 @@
 // Fused LoopVQ decode attention over the packed index cache (sm_100a).
 //
-// Two kernels per call.
+// Three kernels per call, each a programmatic dependent of the one before.
+//
+// vq_lut_kernel: one CTA per (sequence, query head) pair with quantised
+// tokens builds the pair's key lookup table
+//     LUT[e][j] = s*log2(e) * q_j . C_K[j][e][tau]
+// (E x J floats) into the workspace.
 //
 // vq_stream_kernel: a persistent grid (at most one CTA per SM, sixteen warps)
-// over the quantised tokens of every (sequence, query head) pair. All pages
-// of all pairs form one list and CTA c takes the contiguous range
-// [U*c/n, U*(c+1)/n) of it, so every CTA streams the same number of pages and
-// touches one or a few pairs ("segments"). Per segment:
-//   1. The key codebook slice of the pair's kv-head and loop step is staged
-//      into the (empty) histogram window with cp.async while the warps
-//      request their first index blocks (a register ring); the key lookup
-//      table LUT[e][col] = s*log2(e) * q_j . C_K[j][e][tau] (column col holds
-//      group j = col % J) is built from it and the window is zeroed.
-//   2. Streaming, in chunks of kChunkBlocks blocks per warp. Key phase:
-//      lane = slot; byte s of the slot's rotated row is group (lane+s) % J,
-//      held by LUT column lane+s (the LUT repeats its J columns over 64), and
-//      the scores x (log2 units) stay in registers.
-//      The warps' maxima meet at a barrier; the segment's reference maximum
-//      m becomes the integer ceil(max x) so far (when it rises, the histogram
-//      is shifted right by the difference, which is exact in fixed point).
-//      Value phase, lane = slot again: the slot's weight 2^(x - m) <= 1
-//      becomes the integer w = rn(2^(x - m) * 2^kFixBits) and is added, for
-//      each byte s of the slot's rotated value row, to the shared histogram
-//      cell H[idx][(lane + s) % LB] by a 32-bit shared-memory atomic add on
-//      the low word of a 64-bit cell, with the carry added to the high word.
-//      Integer atomics run at full shared-memory rate on sm_100 and need no
-//      turn taking, so all warps update the one histogram concurrently.
-//   3. The histogram, converted to float, is contracted with the value
-//      codebook slice, o_j = sum_e W[e][j] C_V[j][e][tau], and the segment
-//      record (m, l = sum_e W[e][j], o[d]) goes to slot (pair + cta).
+// over the quantised tokens of every pair. All pages of all pairs form one
+// list and CTA c takes the contiguous range [U*c/n, U*(c+1)/n) of it, so
+// every CTA streams the same number of pages and touches one or a few pairs
+// ("segments"). Per segment:
+//   1. The pair's LUT is copied into shared memory with its J columns
+//      repeated over 64 (column c holds group c % J), and the value histogram
+//      H[e][c] (64 columns of 32-bit words) is zeroed.
+//   2. Streaming, in chunks of kChunkBlocks index blocks (LB slots each) per
+//      warp. Key phase, lane = slot: byte s of the slot's rotated K row is
+//      group (lane+s) % J, held by LUT column lane+s, so the lookup address is
+//      one byte permute plus the immediate 4s; the scores x (log2 units) stay
+//      in registers. The warps' maxima and weight sums meet at a barrier,
+//      which fixes the segment's integer reference maximum m (raised to
+//      ceil(max x)) and its fixed-point exponent S. Value phase, lane = slot
+//      again: the slot's weight w = rn(2^(x - m + S)) is added to cell
+//      H[idx][lane + s] for each byte s of its rotated V row by a 32-bit
+//      shared-memory reduction (red.shared.add.u32: integer reductions run
+//      at full shared-memory rate on sm_100, so all warps update the one
+//      histogram without taking turns).
+//      Overflow: every cell is a sum of weights of distinct tokens, so it
+//      never exceeds the total weight of the segment, which the barrier
+//      knows exactly. S starts at kFixMax and is lowered whenever that total
+//      would pass 2^31; m rises when a chunk's maximum passes it. Either
+//      change is an exact right shift of every cell by the bits lost.
+//   3. The histogram, converted to float (W[e][j] = 2^-S sum of the columns
+//      of group j), is contracted with the value codebook slice,
+//      o_j = sum_e W[e][j] C_V[j][e][tau], and the segment record
+//      (m, l = sum_e W[e][j], o[d]) goes to slot (pair + cta).
 //
 // vq_finish_kernel: one CTA per pair scores the bf16 window tokens (prefix +
 // recent), merges them with the pair's segment records (log-sum-exp
 // weights) and writes out and lse.
 //
-// The hot loops address shared memory by absolute shared-window address, so
-// that one byte permute of an index byte gives a complete address: the LUT
-// sits in a 64 KB-aligned window with 256-byte rows (64 columns) and the
-// histogram in the next 64 KB window with 256-byte rows (low words in bytes
-// 0..127 of a row, high words in bytes 128..255). Both windows are placed at run time
-// above the dynamic allocation's base; a CTA whose allocation cannot hold
-// them writes NaN records and flags the call's status word instead of
-// running.
+// The hot loops address shared memory by absolute shared-window address: a
+// byte permute puts an index byte into byte 1 of (lane * 4), and the window
+// base plus 4s is the instruction's immediate offset. That needs the dynamic
+// allocation to start at kSBase, which the host checks before launching (the
+// device's reserved shared memory per block) and every CTA checks again; a
+// CTA that finds another base writes NaN records and flags the status word.
 
 #include <math.h>
 
@@ -59,35 +64,27 @@ constexpr int kThreads = kNW * 32;
 constexpr int kRing = 4;                  // index blocks in registers
 constexpr int kChunkBlocks = 4;           // blocks per warp per chunk (key phase, then value phase)
 constexpr int kPrefetchPages = 4;         // pages a warp asks L2 to fetch ahead of its loads
-constexpr int kFixBits = 30;              // fixed-point weight: w = rn(p * 2^kFixBits), p <= 1
-constexpr float kFixScale = 1073741824.0f;          // 2^kFixBits
-constexpr float kFixInv = 1.0f / 1073741824.0f;     // 2^-kFixBits
+constexpr int kFixMax = 30;               // largest fixed-point exponent: w = rn(2^(x - m) * 2^S)
+constexpr float kMassHigh = 2147483648.0f;  // 2^31: lower S before a segment's total passes this
+constexpr int kMassLandLog2 = 29;         // after lowering S the total sits below 2^29
 constexpr int kFinishThreads = 256;
+constexpr int kLutThreads = 256;          // one thread per centroid
 constexpr int kWinChunk = 9;              // window tokens per warp per round of loads (72 = 8 warps x 9)
 constexpr int kSegmentUnits = 16;         // work units (pages) charged for a segment's setup
+constexpr int kCols = 64;                 // columns of the shared LUT and histogram
 
-// Small area at the start of the dynamic allocation (byte offsets).
-constexpr uint32_t kWmaxOff = 0;                                  // [2][kNW] chunk maxima
-constexpr uint32_t kQsOff = kWmaxOff + 2 * kNW * 4;               // [256] scaled q
-constexpr uint32_t kSmallBytes = kQsOff + 256 * 4;
-constexpr uint32_t kLutBytes = 0x10000u;  // [E][64] floats: column c holds group c % J
-constexpr uint32_t kHistBytes = 0x10000u; // [E][64] words: 32 low, 32 high
-// From any base b with b + kSmallBytes <= 0x10000 the LUT window starts at
-// 0x10000 and the histogram window at 0x20000, so the allocation must reach
-// 0x30000 - b; asking for 0x30000 bytes covers every such base.
-constexpr uint32_t kDynBytes = 0x30000u;
-
-// Groups of a [J][E][C] float codebook slice staged at once into the
-// histogram window: the largest divisor of J whose slice part fits.
-constexpr int stage_groups(int J, int C) {
-  int jc = J;
-  while (jc > 1 && (J % jc != 0 || jc * 256 * C * 4 > static_cast<int>(kHistBytes))) --jc;
-  return jc;
-}
+// Shared memory, by absolute shared-window address. The dynamic allocation
+// starts at kSBase (the reserved shared memory of a block on sm_100).
+constexpr uint32_t kSBase = 0x400u;
+constexpr uint32_t kStatOff = 0;          // [2][kNW][2] per-warp chunk maximum and weight sum
+constexpr uint32_t kSmallBytes = 0x400u;
+constexpr uint32_t kLutAbs = kSBase + kSmallBytes;        // [E][64] floats, 256-byte rows
+constexpr uint32_t kHistAbs = kLutAbs + kE * kCols * 4;   // [E][64] 32-bit words, 256-byte rows
+constexpr uint32_t kDynBytes = kHistAbs + kE * kCols * 4 - kSBase;
 
 // Bits of the status word (see loopvq.h).
-constexpr int kStatusBadPage = 1;
-constexpr int kStatusSharedBase = 2;
+constexpr int kStatusBadPage = LOOPVQ_DECODE_STATUS_BAD_PAGE;
+constexpr int kStatusSharedBase = LOOPVQ_DECODE_STATUS_SHARED_BASE;
 
 struct DecodeParams {
   const uint16_t* q;                // bf16 bits [B][Hq][d]
@@ -101,12 +98,13 @@ struct DecodeParams {
   const uint16_t* win_k;            // bf16 bits [B][Hkv][W][d]
   const uint16_t* win_v;
   float* records;                   // [pairs + n_cta][4 + d]: m, l, -, -, o[d]
+  float* luts;                      // [pairs][E][J] key lookup tables
   int* status;                      // status word (bit flags), never cleared by the kernels
   void* out;
   float* lse;
   int B, Hq, Hkv, ratio, W, Pg, n_pages, max_pages_per_seq, max_seq_len;
   int64_t page_bytes, plane_bytes;
-  int n_cta, out_dtype;
+  int n_cta, out_dtype, log2_bpp;
   float scale_log2;
 };
 
@@ -123,8 +121,13 @@ struct Traits {
 template <int J>
 struct BlockRegs {
   uint32_t w[J / 4];
-  int base;            // first slot of the block inside its page, or -1: no block
-  int valid;           // valid slots in the page (same value in every lane)
+};
+
+// Where a block lives: this lane's row in the K plane (the V plane follows
+// at +plane_bytes) and the number of valid slots (0: no block).
+struct BlockInfo {
+  const uint8_t* row;
+  int nv;
 };
 
 template <int GR>
@@ -143,17 +146,15 @@ __device__ __forceinline__ void load_words(const uint8_t* src, uint32_t* w, int 
   }
 }
 
-// Loads block `blk` of a page's K plane (kv = 0) or V plane (kv = 1): both
-// planes hold rotated slot rows in granules, so lane = slot reads its row.
+// Loads this lane's rotated row of a block whose row starts at `row` (both
+// planes hold rotated slot rows in granules [J/GR][LB][GR]).
 template <int J>
-__device__ __forceinline__ void load_block(const uint8_t* kpl, int64_t plane_bytes, int blk, int kv,
-                                           int lane, BlockRegs<J>& r) {
+__device__ __forceinline__ void load_row(const uint8_t* row, int lane, BlockRegs<J>& r) {
   using T = Traits<J>;
   if (lane < T::LB) {
-    const uint8_t* src = kpl + kv * plane_bytes + blk * T::LB * J + lane * T::GR;
 #pragma unroll
     for (int gi = 0; gi < J / T::GR; ++gi)
-      load_words<T::GR>(src + gi * T::LB * T::GR, r.w + gi * (T::GR / 4), T::GR / 4);
+      load_words<T::GR>(row + gi * T::LB * T::GR, r.w + gi * (T::GR / 4), T::GR / 4);
   } else {
 #pragma unroll
     for (int i = 0; i < T::NWORD; ++i) r.w[i] = 0u;
@@ -179,36 +180,14 @@ __device__ __forceinline__ void load_cw(const float* src, float (&v)[C]) {
   }
 }
 
-// sum_ch a[ch] * b[ch] for C channels held contiguously in shared memory
-// (16-byte aligned when C % 4 == 0).
-template <int C>
-__device__ __forceinline__ float dot_c(const float* a, const float* b) {
-  float v = 0.f;
-  if constexpr (C % 4 == 0) {
-#pragma unroll
-    for (int ch = 0; ch < C; ch += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(a + ch);
-      const float4 y = *reinterpret_cast<const float4*>(b + ch);
-      v = fmaf(x.x, y.x, v);
-      v = fmaf(x.y, y.y, v);
-      v = fmaf(x.z, y.z, v);
-      v = fmaf(x.w, y.w, v);
-    }
-  } else {
-#pragma unroll
-    for (int ch = 0; ch < C; ++ch) v = fmaf(a[ch], b[ch], v);
-  }
-  return v;
-}
-
 // Calls f(std::integral_constant<int, i>) for i = 0 .. N-1 (compile-time i).
-template <int N, typename F, int... I>
+template <typename F, int... I>
 __device__ __forceinline__ void constexpr_for_impl(F&& f, std::integer_sequence<int, I...>) {
   (f(std::integral_constant<int, I>{}), ...);
 }
 template <int N, typename F>
 __device__ __forceinline__ void constexpr_for(F&& f) {
-  constexpr_for_impl<N>(f, std::make_integer_sequence<int, N>{});
+  constexpr_for_impl(f, std::make_integer_sequence<int, N>{});
 }
 
 // ---- shared memory by absolute shared-window address ------------------------
@@ -217,47 +196,16 @@ __device__ __forceinline__ uint32_t smem_addr(const void* ptr) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
 }
 
-// LUT word at address a + OFF: not written while it is read.
-template <int OFF>
-__device__ __forceinline__ float lds_lut(uint32_t a) {
+// Shared word at a + OFF (OFF a compile-time window offset).
+template <uint32_t OFF>
+__device__ __forceinline__ float lds_at(uint32_t a) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(OFF));
   return v;
 }
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-// Histogram update: low word += w; on a carry out of the low word, the high
-// word (128 bytes further along the row) += 1.
-// Histogram updates of four cells by the same weight w: the low words at
-// a0..a3 get w added and their old values come back in o0..o3.
-__device__ __forceinline__ void hist_add4(const uint32_t (&a)[4], uint32_t w, uint32_t (&o)[4]) {
-  asm volatile(
-      "atom.shared.add.u32 %0, [%4], %8;\n"
-      "atom.shared.add.u32 %1, [%5], %8;\n"
-      "atom.shared.add.u32 %2, [%6], %8;\n"
-      "atom.shared.add.u32 %3, [%7], %8;\n"
-      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(w));
-}
-// The carries of those four updates: where an old low word exceeded
-// nw = ~w (the sum wrapped), the high word 128 bytes further along the row
-// gets 1.
-__device__ __forceinline__ void hist_carry4(const uint32_t (&a)[4], const uint32_t (&o)[4],
-                                            uint32_t nw) {
-  asm volatile(
-      "{\n .reg .pred P<4>;\n"
-      " setp.gt.u32 P0, %4, %8;\n setp.gt.u32 P1, %5, %8;\n"
-      " setp.gt.u32 P2, %6, %8;\n setp.gt.u32 P3, %7, %8;\n"
-      " @P0 red.shared.add.u32 [%0+128], 1;\n @P1 red.shared.add.u32 [%1+128], 1;\n"
-      " @P2 red.shared.add.u32 [%2+128], 1;\n @P3 red.shared.add.u32 [%3+128], 1;\n}\n"
-      ::"r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]),
-      "r"(nw));
+template <uint32_t OFF>
+__device__ __forceinline__ void red_at(uint32_t a, uint32_t w) {
+  asm volatile("red.shared.add.u32 [%0+%1], %2;" ::"r"(a), "n"(OFF), "r"(w));
 }
 
 // Quantised-token pages of sequence b.
@@ -426,6 +374,44 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
 }
 
 
+
+// One CTA per pair with quantised tokens: the pair's key lookup table
+// LUT[e][j] = s*log2(e) * sum_ch q[j*C + ch] * C_K[j][e][tau][ch] into
+// luts[pair][e][j]. Thread e owns centroid e; its loads of C_K[j][e][.] are
+// consecutive across the warp.
+template <int J, int C>
+__global__ void __launch_bounds__(kLutThreads) vq_lut_kernel(const DecodeParams p) {
+  constexpr int d = J * C;
+  static_assert(kLutThreads == kE, "one thread per centroid");
+  __shared__ float qs[d];
+  const int pair = blockIdx.x;
+  const int b = pair / p.Hq, hq = pair % p.Hq, hkv = hq / p.ratio;
+  // the streaming kernel may start now; it waits for this grid before it
+  // reads a table
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (seq_pages(p, b) == 0) return;                    // CTA-uniform: no quantised tokens
+  const int e = threadIdx.x;
+  for (int i = e; i < d; i += kLutThreads)
+    qs[i] = bf16_bits_to_float(p.q[static_cast<size_t>(pair) * d + i]) * p.scale_log2;
+  __syncthreads();
+  const float* cbk = p.cb_k + hkv * p.cb_stride_head;  // [J][E][C]
+  float* out = p.luts + (static_cast<size_t>(pair) * kE + e) * J;
+#pragma unroll 1
+  for (int j0 = 0; j0 < J; j0 += 4) {
+    float v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float cw[C];
+      load_cw<C>(cbk + (static_cast<size_t>(j0 + k) * kE + e) * C, cw);
+      float acc = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) acc = fmaf(qs[(j0 + k) * C + ch], cw[ch], acc);
+      v[k] = acc;
+    }
+    *reinterpret_cast<float4*>(out + j0) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
 template <int J, int C>
 __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodeParams p) {
   using T = Traits<J>;
@@ -434,36 +420,21 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   constexpr int KB = kChunkBlocks;                     // blocks per warp per chunk
   constexpr int RS = 4 + d;                            // record floats
   constexpr int EP = kE + 1;                           // padded row of the transposed merged histogram
-  static_assert(J * EP * 4 <= static_cast<int>(kHistBytes), "merged histogram fits the window");
-  static_assert((2 * KB) % kRing == 0, "a chunk's items map onto fixed ring slots");
-  // groups of the key slice staged at once in the (empty) histogram window
-  constexpr int JC = stage_groups(J, C);
-  static_assert(JC >= 1 && J % JC == 0, "staging chunks tile the groups");
-  static_assert(d <= 256, "q fits its buffer");
+  static_assert(KB == kRing, "a chunk's block q lives in ring slot q");
+  static_assert(LB + J - 1 <= kCols, "lookup columns lane + s stay inside the 64 columns");
+  static_assert(J * EP * 4 <= kE * kCols * 4, "merged histogram fits the LUT window");
 
   extern __shared__ __align__(16) unsigned char smem_u8[];
   const uint32_t sbase = smem_addr(smem_u8);
-  float* wmax = reinterpret_cast<float*>(smem_u8 + kWmaxOff);
-  float* qs = reinterpret_cast<float*>(smem_u8 + kQsOff);
-  // the LUT and histogram windows, aligned above the small area
-  const uint32_t lut_abs = (sbase + kSmallBytes + kLutBytes - 1u) & ~(kLutBytes - 1u);
-  const uint32_t hist_abs = lut_abs + kLutBytes;
-  const bool bad_base = hist_abs + kHistBytes > sbase + kDynBytes;
-  float* lut = reinterpret_cast<float*>(smem_u8 + (bad_base ? 0u : lut_abs - sbase));
-  float* stage = reinterpret_cast<float*>(smem_u8 + (bad_base ? 0u : hist_abs - sbase));
+  float* stat = reinterpret_cast<float*>(smem_u8 + kStatOff);
+  float* lut = reinterpret_cast<float*>(smem_u8 + (kLutAbs - kSBase));
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_u8 + (kHistAbs - kSBase));
+  const bool bad_base = sbase != kSBase;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool lane_live = lane < LB;
-  // Byte permutes that put an index byte into byte 1 of these give addresses.
-  // Key lookup s of slot `lane` reads LUT column lane + s (the replicated
-  // columns make the modulo unnecessary): the address of lookup s is
-  // perm(lxb) + 4s. Value update s goes to histogram column (lane + s) % LB.
-  const uint32_t lxb = lut_abs | static_cast<uint32_t>(lane * 4);
-  uint32_t hx[J];
-#pragma unroll
-  for (int s = 0; s < J; ++s) hx[s] = hist_abs | (4u * static_cast<uint32_t>((lane + s) % LB));
-  const int bpp = p.Pg / LB;
-  const uint32_t bpp_magic = 0xFFFFFFFFu / static_cast<uint32_t>(bpp) + 1u;
+  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;   // byte 0 of every table address
+  const int bpp = p.Pg / LB;                           // blocks per page, a power of two
+  const int lbpp = p.log2_bpp;
 
   int b_first;
   long long pre_first;
@@ -483,6 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   int pu_start = static_cast<int>(off % units_b);     // unit offset inside the pair
   long long u = u_lo;
   if (bad_base && tid == 0 && p.status != nullptr) atomicOr(p.status, kStatusSharedBase);
+  bool tables_ready = false;
 
   while (u < u_hi && b < p.B) {
     const int seg_units = static_cast<int>(min(static_cast<long long>(units_b - pu_start), u_hi - u));
@@ -492,7 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
     const int hkv = hq / p.ratio;
     const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
     const int n_vq = max(0, N - p.W);
-    float* rec = p.records + static_cast<size_t>(b * p.Hq + hq + blockIdx.x) * RS;
+    const int pair = b * p.Hq + hq;
+    float* rec = p.records + static_cast<size_t>(pair + blockIdx.x) * RS;
     if (bad_base) {
       if (tid == 0) {
         rec[0] = NAN;
@@ -504,34 +477,29 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         rec[1] = 0.f;
       }
     } else {
-      const float* cbk = p.cb_k + hkv * p.cb_stride_head;
-      const uint16_t* qp = p.q + (static_cast<size_t>(b) * p.Hq + hq) * d;
-      __syncthreads();                                 // previous segment done with LUT, histogram, q
-      // the first chunk of the key slice goes out before anything that waits
-      for (int i = tid * 4; i < JC * kE * C; i += kThreads * 4) cp_async16(stage + i, cbk + i);
+      __syncthreads();                                 // previous segment done with LUT and histogram
       const float* cbv = p.cb_v + hkv * p.cb_stride_head;
       if (warp == kNW - 1) {                           // the value slice, into L2 for the contraction
         constexpr uint32_t kSlice = kE * J * C * 4, kPiece = kSlice / 32;
         static_assert(kSlice % (32 * 16) == 0, "prefetch pieces are 16-byte multiples");
         prefetch_l2_bulk(reinterpret_cast<const char*>(cbv) + lane * kPiece, kPiece);
       }
-      const float qv = (tid < d) ? bf16_bits_to_float(qp[tid]) * p.scale_log2 : 0.f;
 
-      // ---- this warp's pages and the index ring --------------------------------
-      // warp w streams the segment's pages pg_lo + w + k*kNW (k = 0, 1, ..), each
+      // ---- this warp's pages and blocks ----------------------------------------
+      // Warp w streams the segment's pages pg_lo + w + k*kNW (k = 0, 1, ..), each
       // as bpp blocks; its t-th block is block t % bpp of its page t / bpp.
-      // Chunk ch holds blocks [ch*KB, (ch+1)*KB) of every warp; its items are
-      // the KB key blocks, then the same KB value blocks.
+      // Chunk ch holds blocks [ch*KB, (ch+1)*KB) of every warp: their key rows,
+      // then their value rows.
       const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
       const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages_per_seq;
       auto pages_of = [&](int w) { return (pg_hi > pg_lo + w) ? (pg_hi - pg_lo - w + kNW - 1) / kNW : 0; };
       const int my_first = pg_lo + warp;
       const int n_my_pages = pages_of(warp);
-      const int n_blocks = n_my_pages * bpp;
-      const int n_chunks = (pages_of(0) * bpp + KB - 1) / KB;   // CTA-uniform (warp 0 has the most)
-      int i0 = 0;                                      // page-table window: pages [i0, i0 + 64)
+      const int n_blocks = n_my_pages << lbpp;
+      const int n_chunks = ((pages_of(0) << lbpp) + KB - 1) / KB;   // CTA-uniform (warp 0 has the most)
+      int i0 = 0;                                      // page-table window: this warp's pages [i0, i0 + 64)
       auto bt_entry = [&](int i) -> int { return (i < n_my_pages) ? bt[my_first + i * kNW] : -1; };
-      int bt_cur = bt_entry(lane);                     // requested now, used after the slice lands
+      int bt_cur = bt_entry(lane);
       int bt_nxt = bt_entry(32 + lane);
       // L2 prefetch of pages [k0, k1) of this warp's list
       auto prefetch_pages = [&](int k0, int k1) {
@@ -545,169 +513,150 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
                            static_cast<uint32_t>(p.page_bytes));
       };
       BlockRegs<J> ring[kRing];
-#pragma unroll
-      for (int k = 0; k < kRing; ++k) ring[k].base = -1;
-      // a cleared block keeps whatever bytes it held: every byte value
-      // addresses a valid row, and base = -1 masks and skips it
-      auto issue = [&](int i, BlockRegs<J>& r) {
-        const int ch = i / (2 * KB);
-        const int pos = i - ch * 2 * KB;
-        const int kv = pos >= KB ? 1 : 0;
-        const int t = ch * KB + (pos - kv * KB);
-        if (pos == 0) {                                  // first item of a chunk (warp-uniform)
-          const int kmin = static_cast<int>(__umulhi(static_cast<uint32_t>(ch * KB), bpp_magic));
-          if (kmin >= i0 + 32) {                         // slide the page-table window
-            bt_cur = bt_nxt;
-            i0 += 32;
-            bt_nxt = bt_entry(i0 + 32 + lane);
-          }
-          const int knext = static_cast<int>(__umulhi(static_cast<uint32_t>((ch + 1) * KB), bpp_magic));
-          prefetch_pages(kmin + kPrefetchPages, knext + kPrefetchPages);
-        }
-        if (t >= n_blocks) {                             // warp-uniform
-          r.base = -1;
-          return;
-        }
-        const int pi = static_cast<int>(__umulhi(static_cast<uint32_t>(t), bpp_magic));
-        const int blk = t - pi * bpp;
+      BlockInfo info[KB];
+      // Locates block t of this warp (its key row is loaded by the caller).
+      auto locate = [&](int t, BlockInfo& bi) {
+        bi.nv = 0;
+        if (t >= n_blocks) return;                     // warp-uniform
+        const int pi = t >> lbpp, blk = t & (bpp - 1);
         const int src = (pi - i0 < 32) ? bt_cur : bt_nxt;
         const int phys = __shfl_sync(0xffffffffu, src, (pi - i0) & 31);
-        const int pg = my_first + pi * kNW;
-        r.valid = min(p.Pg, n_vq - pg * p.Pg);
-        r.base = blk * LB;
-        if (phys < 0 || phys >= p.n_pages) {             // a page-table entry outside the pool
+        if (phys < 0 || phys >= p.n_pages) {           // a page-table entry outside the pool
           if (lane == 0 && p.status != nullptr) atomicOr(p.status, kStatusBadPage);
-          r.base = -1;
           return;
         }
-        if (r.base >= r.valid) {                         // past the sequence's last token
-          r.base = -1;
-          return;
+        const int pg = my_first + pi * kNW;
+        bi.nv = max(0, min(LB, n_vq - pg * p.Pg - blk * LB));
+        bi.row = pool_h + static_cast<int64_t>(phys) * p.page_bytes + blk * (LB * J) + lane * T::GR;
+      };
+      // the key rows of chunk ch into the ring (and their locations into info)
+      auto issue_keys = [&](int ch) {
+        const int kmin = (ch * KB) >> lbpp;            // first page of the chunk
+        if (kmin >= i0 + 32) {                         // slide the page-table window
+          bt_cur = bt_nxt;
+          i0 += 32;
+          bt_nxt = bt_entry(i0 + 32 + lane);
         }
-        load_block<J>(pool_h + static_cast<int64_t>(phys) * p.page_bytes, p.plane_bytes, blk, kv, lane,
-                      r);
+        prefetch_pages(kmin + kPrefetchPages, (((ch + 1) * KB) >> lbpp) + kPrefetchPages);
+      };
+      auto issue_key = [&](int ch, int q) {
+        locate(ch * KB + q, info[q]);
+        if (info[q].nv > 0) load_row<J>(info[q].row, lane, ring[q]);
+      };
+      auto issue_value = [&](int q) {
+        if (info[q].nv > 0) load_row<J>(info[q].row + p.plane_bytes, lane, ring[q]);
       };
 
-      // ---- key LUT from the key slice staged in the histogram window ----------
-      if (tid < d) qs[tid] = qv;
-#pragma unroll 1
-      for (int j0 = 0; j0 < J; j0 += JC) {
-        if (j0 > 0) {
-          __syncthreads();                             // previous chunk consumed
-          const float* src = cbk + static_cast<size_t>(j0) * kE * C;
-          for (int i = tid * 4; i < JC * kE * C; i += kThreads * 4) cp_async16(stage + i, src + i);
-        }
-        cp_async_wait_all();
-        __syncthreads();
-        if (j0 == 0) {                                 // the page table has landed: first index blocks
-          prefetch_pages(0, kPrefetchPages);
+      // ---- first key rows, then the pair's LUT and a zero histogram --------------
+      prefetch_pages(0, kPrefetchPages);
+      issue_keys(0);
 #pragma unroll
-          for (int k = 0; k < kRing; ++k) issue(k, ring[k]);
-        }
-        // item = (tile of 32 rows, step): lane -> row tile*32 + lane, group
-        // j0 + (step + lane) % JC, so the lanes' table stores hit distinct banks
-#pragma unroll 4
-        for (int it = warp; it < (kE / 32) * JC; it += kNW) {
-          const int e = (it / JC) * 32 + lane, jj = (it % JC + lane) % JC, j = j0 + jj;
-          const float v = dot_c<C>(qs + j * C, stage + (static_cast<size_t>(jj) * kE + e) * C);
-#pragma unroll
-          for (int c = j; c < 64; c += J) lut[e * 64 + c] = v;   // every column holding group j
-        }
+      for (int q = 0; q < KB; ++q) issue_key(0, q);
+      if (!tables_ready) {                             // the LUT kernel's tables are complete
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        tables_ready = true;
       }
-      __syncthreads();                                 // LUT complete; staging area free
-      for (uint32_t a = hist_abs + 16u * tid; a < hist_abs + kHistBytes; a += 16u * kThreads)
-        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
-      __syncthreads();                                 // histogram zero
+      {
+        const float4* src = reinterpret_cast<const float4*>(p.luts + static_cast<size_t>(pair) * kE * J);
+        for (int f = tid; f < kE * J / 4; f += kThreads) {
+          const float4 v = __ldcg(src + f);
+          const int e = f / (J / 4), c0 = (f - e * (J / 4)) * 4;
+          for (int c = c0; c + 4 <= kCols; c += J) *reinterpret_cast<float4*>(lut + e * kCols + c) = v;
+        }
+        for (int i = tid * 4; i < kE * kCols; i += kThreads * 4)
+          *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncthreads();                                 // LUT and histogram ready
 
       // ---- stream -------------------------------------------------------------
-      auto key_scores = [&](const BlockRegs<J>& r) -> float {
-        if (r.base < 0) return -INFINITY;              // warp-uniform
-        float xa[4] = {0.f, 0.f, 0.f, 0.f};
+      auto key_score = [&](const BlockRegs<J>& r, int nv) -> float {
+        if (nv <= 0) return -INFINITY;                 // warp-uniform
         uint32_t ad[J];
 #pragma unroll
-        for (int s = 0; s < J; ++s) ad[s] = __byte_perm(r.w[s >> 2], lxb, 0x7604u | (uint32_t(s & 3) << 4));
-        constexpr_for<J>([&](auto S) { xa[S.value & 3] += lds_lut<4 * S.value>(ad[S.value]); });
-        const bool valid = lane_live && (r.base + lane) < r.valid;
-        return valid ? (xa[0] + xa[1]) + (xa[2] + xa[3]) : -INFINITY;
+        for (int s = 0; s < J; ++s) ad[s] = __byte_perm(r.w[s >> 2], lane4, 0x7604u | (uint32_t(s & 3) << 4));
+        float xa[4] = {0.f, 0.f, 0.f, 0.f};
+        constexpr_for<J>([&](auto S) { xa[S.value & 3] += lds_at<kLutAbs + 4u * S.value>(ad[S.value]); });
+        return lane < nv ? (xa[0] + xa[1]) + (xa[2] + xa[3]) : -INFINITY;
       };
       // histogram updates of one value block, lane = slot: the slot's weight
-      // w = rn(2^(x - m) * 2^kFixBits) goes to row idx_V[slot][j] of column
-      // (lane + s) % LB for each byte s of its rotated row; carries out of a low
-      // word go to its high word
-      auto value_pass = [&](const BlockRegs<J>& r, float x, float m) {
-        if (r.base < 0) return;                        // warp-uniform
-        if constexpr (LB < 32) {
-          if (!lane_live) return;
-        }
-        uint32_t w = __float2uint_rn(fast_exp2(x - m) * kFixScale);   // 0 for x = -inf
-        w = min(w, 1u << kFixBits);
-        const uint32_t nw = ~w;
-        uint32_t a[4], o[4];
+      // w = rn(2^(x - m + S)) goes to cell [idx][lane + s] for each byte s of its
+      // rotated value row (w = 0 for an invalid slot)
+      auto value_pass = [&](const BlockRegs<J>& r, int nv, float x, float mS) {
+        if (nv <= 0) return;                           // warp-uniform
+        const uint32_t w = __float2uint_rn(fast_exp2(x - mS));
+        uint32_t ad[J];
 #pragma unroll
-        for (int i = 0; i < J / 4; ++i) {
-          uint32_t an[4], on[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) an[k] = __byte_perm(r.w[i], hx[4 * i + k], 0x7604u | (uint32_t(k) << 4));
-          hist_add4(an, w, on);
-          if (i > 0) hist_carry4(a, o, nw);            // the previous four, whose old words are back
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            a[k] = an[k];
-            o[k] = on[k];
-          }
-        }
-        hist_carry4(a, o, nw);
+        for (int s = 0; s < J; ++s) ad[s] = __byte_perm(r.w[s >> 2], lane4, 0x7604u | (uint32_t(s & 3) << 4));
+        constexpr_for<J>([&](auto S) { red_at<kHistAbs + 4u * S.value>(ad[S.value], w); });
       };
-      // exact rescale of the 64-bit cells by 2^-sh when the reference maximum rises
+      // every cell >>= sh (an exact rescale of the fixed-point weights)
       auto rescale = [&](int sh) {
-        for (int cell = tid; cell < kE * 32; cell += kThreads) {
-          const uint32_t ad = hist_abs + (static_cast<uint32_t>(cell >> 5) << 8) +
-                              (static_cast<uint32_t>(cell & 31) << 2);
-          uint32_t lo = lds_u32(ad), hi = lds_u32(ad + 128u);
-          if (sh >= 64) {
-            lo = 0u;
-            hi = 0u;
-          } else if (sh >= 32) {
-            lo = hi >> (sh - 32);
-            hi = 0u;
+        for (int i = tid * 4; i < kE * kCols; i += kThreads * 4) {
+          uint4 v = *reinterpret_cast<uint4*>(hist + i);
+          if (sh >= 32) {
+            v = make_uint4(0u, 0u, 0u, 0u);
           } else {
-            lo = __funnelshift_r(lo, hi, sh);
-            hi >>= sh;
+            v.x >>= sh; v.y >>= sh; v.z >>= sh; v.w >>= sh;
           }
-          sts_u32(ad, lo);
-          sts_u32(ad + 128u, hi);
+          *reinterpret_cast<uint4*>(hist + i) = v;
         }
       };
 
       float m_cur = -INFINITY;                         // integer reference maximum (CTA-uniform)
+      int S = kFixMax;                                 // fixed-point exponent (CTA-uniform)
+      float mass = 0.f;                                // sum of weights so far, units of 2^(m_cur) (CTA-uniform)
 #pragma unroll 1
       for (int ch = 0; ch < n_chunks; ++ch) {
-        const int ib = ch * 2 * KB;
         float xs[KB];
         float cm = -INFINITY;
 #pragma unroll
         for (int q = 0; q < KB; ++q) {                 // key phase
-          xs[q] = key_scores(ring[q % kRing]);
+          xs[q] = key_score(ring[q], info[q].nv);
           cm = fmaxf(cm, xs[q]);
-          issue(ib + q + kRing, ring[q % kRing]);
+          issue_value(q);
         }
         cm = warp_max(cm);
-        if (lane == 0) wmax[(ch & 1) * kNW + warp] = cm;
-        __syncthreads();                               // every warp's chunk maximum
-        float cmax = (lane < kNW) ? wmax[(ch & 1) * kNW + lane] : -INFINITY;
-        cmax = warp_max(cmax);
+        float ps = 0.f;                                // sum of 2^(x - cm) over this warp's slots
+        if (cm != -INFINITY) {                         // warp-uniform
+#pragma unroll
+          for (int q = 0; q < KB; ++q) ps += fast_exp2(xs[q] - cm);   // 0 for x = -inf
+          ps = warp_sum(ps);
+        }
+        float* st = stat + (ch & 1) * 2 * kNW;
+        if (lane == 0) {
+          st[2 * warp] = cm;
+          st[2 * warp + 1] = ps;
+        }
+        __syncthreads();                               // every warp's chunk maximum and sum
+        const float cmw = (lane < kNW) ? st[2 * lane] : -INFINITY;
+        const float cmax = warp_max(cmw);
         if (cmax != -INFINITY) {                       // CTA-uniform
           const float m_new = fmaxf(m_cur, ceilf(cmax));
-          if (m_cur != -INFINITY && m_new > m_cur) {   // earlier chunks' weights shrink by 2^-(m_new - m_cur)
-            rescale(static_cast<int>(fminf(m_new - m_cur, 64.f)));
+          const float psw = (lane < kNW && cmw != -INFINITY) ? st[2 * lane + 1] * fast_exp2(cmw - m_new) : 0.f;
+          const float add = warp_sum(psw);             // the chunk's weights, units of 2^m_new
+          const float kept = (m_cur == -INFINITY) ? 0.f : mass * fast_exp2(m_cur - m_new);
+          const float total = kept + add;
+          int S_new = S;
+          if (ldexpf(total, S) + static_cast<float>(kThreads * KB) > kMassHigh) {
+            int ex;
+            frexpf(total, &ex);                        // total < 2^ex
+            S_new = min(S, kMassLandLog2 - ex);
+          }
+          const int sh = ((m_cur == -INFINITY) ? 0 : static_cast<int>(m_new - m_cur)) + (S - S_new);
+          if (m_cur != -INFINITY && sh > 0) {          // earlier weights shrink by 2^-sh
+            rescale(sh);
             __syncthreads();
           }
           m_cur = m_new;
+          S = S_new;
+          mass = total;
         }
+        const float mS = m_cur - static_cast<float>(S);
 #pragma unroll
         for (int q = 0; q < KB; ++q) {                 // value phase
-          if (m_cur != -INFINITY) value_pass(ring[(KB + q) % kRing], xs[q], m_cur);   // CTA-uniform
-          issue(ib + KB + q + kRing, ring[(KB + q) % kRing]);
+          if (m_cur != -INFINITY) value_pass(ring[q], info[q].nv, xs[q], mS);   // CTA-uniform
+          if (q == 0) issue_keys(ch + 1);
+          issue_key(ch + 1, q);
         }
       }
       __syncthreads();                                 // every update landed
@@ -719,29 +668,19 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           rec[1] = 0.f;
         }
       } else {
-        // W[e][j]: lane = column, rows warp + kNW*k; replicas of a group are summed
+        // W[e][j] = 2^-S * sum of the columns c = j (mod J): lane = group, rows warp + kNW*k
         constexpr int NR = kE / kNW;                   // rows per warp
-        float wv[NR];
+        const float inv = ldexpf(1.f, -S);
+        float* wt = lut;                               // transposed, padded: wt[j*EP + e]
 #pragma unroll
         for (int k = 0; k < NR; ++k) {
           const int e = warp + kNW * k;
-          float v = 0.f;
-          if (lane_live) {
-            const uint32_t ad = hist_abs + (static_cast<uint32_t>(e) << 8) + 4u * lane;
-            const uint32_t lo = lds_u32(ad), hi = lds_u32(ad + 128u);
-            v = (__uint2float_rn(hi) * 4294967296.0f + __uint2float_rn(lo)) * kFixInv;
+          if (lane < J) {
+            unsigned long long v = 0ull;
+#pragma unroll
+            for (int c = lane; c < kCols; c += J) v += hist[e * kCols + c];
+            wt[lane * EP + e] = static_cast<float>(v) * inv;
           }
-#pragma unroll
-          for (int o = (T::R / 2) * J; o >= J; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-          wv[k] = v;
-        }
-        __syncthreads();                               // every histogram word read
-        // transposed, padded: wt[j*EP + e] (lanes of a row and of a column hit distinct banks)
-        float* wt = stage;
-#pragma unroll
-        for (int k = 0; k < NR; ++k) {
-          const int e = warp + kNW * k;
-          if (lane < J) wt[lane * EP + e] = wv[k];
         }
         __syncthreads();
         // o[j*C + ch] = sum_e W[e][j] C_V[j][e][ch]: warp -> groups, lane -> rows lane + 32 i
@@ -791,6 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       } while (b < p.B && u < u_hi && (units_b = pair_units(seq_pages(p, b))) == 0);
     }
   }
+  if (!tables_ready) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // One CTA per (sequence, query head): the bf16 window partial and the merge
@@ -888,11 +828,20 @@ __global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeP
 
 template <typename K>
 loopvq_status set_smem(K kernel, size_t smem, std::atomic<uint64_t>& configured) {
-  // The attribute belongs to (function, device); remember which devices have it.
+  // The attribute belongs to (function, device); remember which devices have
+  // it. The streaming kernel's shared-memory addresses assume its dynamic
+  // allocation starts at kSBase: right after the block's reserved shared
+  // memory, with no static shared memory before it.
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LOOPVQ_ERR_CUDA;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
   if (bit == 0 || !(configured.load(std::memory_order_relaxed) & bit)) {
+    int reserved = -1;
+    if (cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+      return LOOPVQ_ERR_CUDA;
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+    if (reserved != static_cast<int>(kSBase) || fa.sharedSizeBytes != 0) return LOOPVQ_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return LOOPVQ_ERR_CUDA;
@@ -901,36 +850,56 @@ loopvq_status set_smem(K kernel, size_t smem, std::atomic<uint64_t>& configured)
   return LOOPVQ_OK;
 }
 
-template <int J, int C>
-loopvq_status launch_vq(const DecodeParams& p, cudaStream_t st, bool run_stream) {
-  static_assert(kDynBytes <= 227 * 1024, "streaming kernel shared memory above 227 KB");
-  if (run_stream) {
-    static std::atomic<uint64_t> configured{0};
-    if (set_smem(vq_stream_kernel<J, C>, kDynBytes, configured) != LOOPVQ_OK) return LOOPVQ_ERR_CUDA;
-    vq_stream_kernel<J, C><<<p.n_cta, kThreads, kDynBytes, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return LOOPVQ_ERR_CUDA;
-  }
-  // programmatic dependent launch: the finish kernel's CTAs may start while
-  // the streaming kernel's last CTAs still run (griddepcontrol.wait inside)
+// Launches `kernel` as a programmatic dependent of the previous kernel on
+// the stream: its CTAs may start while that kernel's last CTAs still run
+// (griddepcontrol.wait inside orders the reads that need its results).
+template <typename K>
+loopvq_status launch_dependent(K kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                               const DecodeParams& p) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.B * p.Hq));
-  cfg.blockDim = dim3(kFinishThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, vq_finish_kernel<J, C>, p) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LOOPVQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+}
+
+template <int J, int C>
+loopvq_status launch_vq(const DecodeParams& p, cudaStream_t st, bool run_stream) {
+  static_assert(kDynBytes <= 227 * 1024, "streaming kernel shared memory above 227 KB");
+  const unsigned pairs = static_cast<unsigned>(p.B * p.Hq);
+  if (run_stream) {
+    static std::atomic<uint64_t> configured{0};
+    const loopvq_status s = set_smem(vq_stream_kernel<J, C>, kDynBytes, configured);
+    if (s != LOOPVQ_OK) return s;
+    vq_lut_kernel<J, C><<<pairs, kLutThreads, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return LOOPVQ_ERR_CUDA;
+    const loopvq_status s2 =
+        launch_dependent(vq_stream_kernel<J, C>, static_cast<unsigned>(p.n_cta), kThreads, kDynBytes, st, p);
+    if (s2 != LOOPVQ_OK) return s2;
+  }
+  return launch_dependent(vq_finish_kernel<J, C>, pairs, kFinishThreads, 0, st, p);
 }
 
 }  // namespace
 
+size_t decode_lut_bytes(int pairs, int J) {
+  return static_cast<size_t>(pairs) * kE * J * sizeof(float);
+}
+
 loopvq_status launch_decode(const DecodeArgs& a) {
   const Geometry& g = *a.geo;
   const int gamma = a.loop_step / g.g, tau = a.loop_step % g.g;
+  const int bpp = g.Pg / g.LB;
+  int log2_bpp = 0;
+  while ((1 << log2_bpp) < bpp) ++log2_bpp;
+  if ((1 << log2_bpp) != bpp) return LOOPVQ_ERR_UNSUPPORTED;
   DecodeParams p{};
   p.q = static_cast<const uint16_t*>(a.q);
   p.pool_lg = a.pool + a.layer * g.pool_stride_layer + gamma * g.pool_stride_group;
@@ -944,8 +913,13 @@ loopvq_status launch_decode(const DecodeArgs& a) {
   p.seq_lens = a.seq_lens;
   p.win_k = static_cast<const uint16_t*>(a.win_k);
   p.win_v = static_cast<const uint16_t*>(a.win_v);
-  p.status = static_cast<int*>(a.workspace);
-  p.records = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + kStatusBytes);
+  // workspace: status word, segment records, key lookup tables
+  char* ws = static_cast<char*>(a.workspace);
+  const size_t pairs = static_cast<size_t>(a.batch) * g.Hq;
+  p.status = reinterpret_cast<int*>(ws);
+  p.records = reinterpret_cast<float*>(ws + kStatusBytes);
+  p.luts = reinterpret_cast<float*>(ws + kStatusBytes +
+                                    (pairs + kMaxStreamCtas) * (4 + static_cast<size_t>(g.d)) * sizeof(float));
   p.out = a.out;
   p.lse = a.lse;
   p.B = a.batch;
@@ -961,6 +935,7 @@ loopvq_status launch_decode(const DecodeArgs& a) {
   p.plane_bytes = g.plane_bytes;
   p.n_cta = a.n_cta;
   p.out_dtype = a.out_dtype;
+  p.log2_bpp = log2_bpp;
   p.scale_log2 = a.sm_scale * kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(a.stream);
   const bool run = a.n_cta > 0;

@@ -29,8 +29,12 @@ int max_decode_splits(int pairs, int pages);
 constexpr int kMaxStreamCtas = 256;
 
 // Bytes at the start of the decode workspace that hold the status word (an
-// int32 of flag bits); the segment records follow.
+// int32 of flag bits); the segment records follow, then one key lookup table
+// of E x J floats per (sequence, query head) pair.
 constexpr size_t kStatusBytes = 256;
+
+// Bytes of the key lookup tables of `pairs` pairs with J channel groups.
+size_t decode_lut_bytes(int pairs, int J);
 
 // Number of multiprocessors of the current device (cached per device).
 // Returns 0 and sets *err when the runtime fails.

@@ -73,6 +73,7 @@ def test_layout_rate_and_sizes(c, g, bits):
     (dict(chan_group=2), B.LOOPVQ_ERR_UNSUPPORTED),         # J = 64 > 32
     (dict(loop_group=8, n_loops=8, chan_group=8), B.LOOPVQ_ERR_UNSUPPORTED),  # D = 64
     (dict(page_tokens=48), B.LOOPVQ_ERR_UNSUPPORTED),       # not a multiple of LB = 32
+    (dict(page_tokens=96), B.LOOPVQ_ERR_UNSUPPORTED),       # 3 blocks of LB = 32: not a power of two
     (dict(prefix_tokens=200, recent_tokens=100), B.LOOPVQ_ERR_UNSUPPORTED),
 ])
 def test_layout_rejects(kw, status):
@@ -171,10 +172,12 @@ def test_kmeans_step_rejects_before_launch():
 def test_workspace_bytes_formula():
     cfg = _cfg()
     # a 256-byte status area, then one record (m, l, 2 spare, o[d]) of float32
-    # per (pair, streaming CTA) slot: pairs + 256 slots
+    # per (pair, streaming CTA) slot: pairs + 256 slots, then one key lookup
+    # table of 256 x J float32 per pair
     n = L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64)
     rec = 4 * (4 + cfg.head_dim)
-    assert n == 256 + rec * (2 * cfg.n_q_heads + 256)
+    pairs, J = 2 * cfg.n_q_heads, cfg.head_dim // cfg.chan_group
+    assert n == 256 + rec * (pairs + 256) + pairs * 256 * J * 4
     # more sequences need more records
     assert L.loopvq_decode_workspace_bytes(cfg, 4, 72 + 5 * 64) > n
     assert L.loopvq_decode_workspace_bytes(cfg, 0, 10) == 0
