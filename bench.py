@@ -40,7 +40,7 @@ def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="loopvq", choices=["loopvq", "reference"])
     ap.add_argument("--config", default="long32k")
     ap.add_argument("--no-extras", action="store_true",
@@ -283,6 +283,8 @@ class Workload:
                                     self.evict_slots, self.pool, stream=stream)
 
     def launches_per_step(self):
+        """Kernels per step: two per decode call (the pair kernel, the
+        streaming kernel) and one per eviction encode."""
         s = self.shape
         return s.n_loops * s.n_layers * 2 + s.n_layers * s.G * 2
 
@@ -387,6 +389,177 @@ def bf16_comparison(shape, device, reps=20):
     torch.cuda.empty_cache()
     return {"us_per_call": us, "gbps": nbytes / us / 1e3, "bytes_per_call": nbytes,
             "shape": f"B={B} Hkv={H} d={d} N={N} bf16 K/V"}
+
+
+def alg_bytes_per_call(shape, seq_lens) -> int:
+    """Bytes one decode call must move: the packed K and V indices of every
+    quantised token of every (sequence, query head), the bf16 window tokens,
+    the loop-step slice of the K and V codebooks of every kv-head, and q,
+    out (bf16) and lse."""
+    s = shape
+    n_vq = sum(max(0, n - s.window) for n in seq_lens)
+    n_win = sum(min(n, s.window) for n in seq_lens)
+    idx = 2 * s.J * n_vq * s.n_q_heads
+    win = 2 * n_win * s.head_dim * 2 * s.n_kv_heads
+    cb = 2 * 256 * s.head_dim * 4 * s.n_kv_heads
+    io = len(seq_lens) * s.n_q_heads * (s.head_dim * 2 * 2 + 4)
+    return idx + win + cb + io
+
+
+def encoded_layers(shape, n_layers, seq_lens, gammas, device, chunk=1 << 18):
+    """A pool of `n_layers` layers whose indices the GPU encoder wrote from the
+    synthetic loop-group K/V of the shape (codebooks fitted by Lloyd on
+    samples of the same distribution), for the loop groups `gammas`. Returns
+    (config, pool, codebooks, block table)."""
+    import torch
+
+    import sub_bit_vq_b200 as L
+    from synthetic import block_tables, codebooks_for_layer, loop_group_kv
+
+    s = shape
+    B = len(seq_lens)
+    bt, n_pages = block_tables(s, B, seq_lens)
+    cfg = L.LoopVQConfig(n_layers=n_layers, n_kv_heads=s.n_kv_heads, n_q_heads=s.n_q_heads,
+                         head_dim=s.head_dim, n_loops=s.n_loops, loop_group=s.loop_group,
+                         chan_group=s.chan_group, n_pages=n_pages, max_batch=B,
+                         max_pages_per_seq=bt.shape[1], prefix_tokens=s.prefix,
+                         recent_tokens=s.recent, page_tokens=s.page_tokens)
+    pool = torch.zeros(L.loopvq_cache_layout(cfg)["pool_bytes"], dtype=torch.uint8, device=device)
+    cb = torch.empty(n_layers, s.n_kv_heads, s.G, 2, s.loop_group, s.J, 256, s.chan_group,
+                     device=device)
+    btd = bt.to(device)
+    slots = []
+    for b, n in enumerate(seq_lens):
+        v = torch.arange(max(0, n - s.window), device=device)
+        slots.append(btd[b][v // s.page_tokens].long() * s.page_tokens + v % s.page_tokens)
+    slots = torch.cat(slots)
+    total = int(slots.numel())
+    for l in range(n_layers):
+        cb[l] = codebooks_for_layer(s, l, device=device, n_samples=1024, iters=10)
+        for gamma in gammas:
+            for kv in range(2):
+                for k, c0 in enumerate(range(0, total, chunk)):
+                    n = min(chunk, total - c0)
+                    x = loop_group_kv(s, l, gamma, kv, n, device=device, stream=k)
+                    L.loopvq_encode(cfg, l, gamma, kv, x, None, cb, slots[c0:c0 + n], pool)
+                    del x
+    torch.cuda.synchronize()
+    return cfg, pool, cb, btd
+
+
+def time_calls(calls, reps, warm=3):
+    """Per-call device times (CUDA events around each call, queue kept full)
+    and the back-to-back average of `reps` calls without events, in µs.
+    `calls` is a list of callables taking a stream handle; they rotate."""
+    import torch
+    st = torch.cuda.current_stream()
+    for i in range(warm):
+        calls[i % len(calls)](st.cuda_stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    torch.cuda.synchronize()
+    for i in range(reps):
+        ev[i][0].record(st)
+        calls[i % len(calls)](st.cuda_stream)
+        ev[i][1].record(st)
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) * 1e3 for a, b in ev]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for i in range(reps):
+        calls[i % len(calls)](st.cuda_stream)
+    e1.record(st)
+    torch.cuda.synchronize()
+    return per, e0.elapsed_time(e1) * 1e3 / reps
+
+
+def decode_row(shape, seq_lens, n_layers, loop_steps, device, peak, l2_bytes, rotate_seqs=None):
+    """One measured decode configuration: the LoopVQ call (layers, or
+    sequence subsets, rotate so that the calls of a round move at least 4x
+    the L2 size) and the same-shape bf16-KV kernel beside it."""
+    import torch
+
+    import sub_bit_vq_b200 as L
+    from synthetic import queries, window_kv
+
+    s = shape
+    B = len(seq_lens)
+    gammas = sorted({t // s.loop_group for t in loop_steps})
+    all_lens = seq_lens if rotate_seqs is None else seq_lens * rotate_seqs
+    cfg, pool, cb, bt = encoded_layers(s, n_layers, all_lens, gammas, device)
+    nb = len(all_lens)
+    sl_all = torch.tensor(all_lens, dtype=torch.int32, device=device)
+    max_len = max(seq_lens)
+    wsb = L.loopvq_decode_workspace_bytes(cfg, B, max_len)
+    alg = alg_bytes_per_call(s, seq_lens)
+    n_rot = max(1, -(-4 * l2_bytes // alg))
+    calls = []
+    keep = []
+    for k in range(n_rot):
+        l = k % n_layers
+        r = (k // n_layers) % (nb // B)
+        t = loop_steps[k % len(loop_steps)]
+        q = queries(s, l, t, batch=nb, device=device)[r * B:(r + 1) * B].contiguous()
+        wk = window_kv(s, l, t, 0, batch=nb, device=device)[r * B:(r + 1) * B].contiguous()
+        wv = window_kv(s, l, t, 1, batch=nb, device=device)[r * B:(r + 1) * B].contiguous()
+        out = torch.empty(B, s.n_q_heads, s.head_dim, dtype=torch.bfloat16, device=device)
+        lse = torch.empty(B, s.n_q_heads, device=device)
+        ws = torch.empty(wsb // 4 + 4, device=device)
+        btr, slr = bt[r * B:(r + 1) * B], sl_all[r * B:(r + 1) * B]
+        keep.append((q, wk, wv, out, lse, ws, btr, slr))
+
+        def call(stream, l=l, t=t, a=keep[-1]):
+            L.loopvq_decode_attn(cfg, l, t, a[0], pool, cb, a[6], a[7], a[1], a[2], a[3], a[5],
+                                 max_len, lse=a[4], stream=stream)
+        calls.append(call)
+    per, avg = time_calls(calls, reps=max(30, n_rot))
+    p10, med, p90 = call_percentiles(per)
+    row = {"batch": B, "context": max_len, "us_per_call": med, "us_p10_median_p90": [p10, med, p90],
+           "us_back_to_back": avg, "alg_bytes_per_call": alg, "gbps": alg / med / 1e3,
+           "frac_of_measured_hbm": alg / med / 1e3 / peak, "rotation": n_rot}
+    del keep, calls, pool
+    torch.cuda.empty_cache()
+    # the same-shape bf16-KV kernel: distinct K/V per rotation
+    n_rot_b = max(1, -(-4 * l2_bytes // (2 * B * s.n_kv_heads * max_len * s.head_dim * 2)))
+    ks = [torch.randn(B, s.n_kv_heads, max_len, s.head_dim, device=device, dtype=torch.bfloat16)
+          for _ in range(n_rot_b)]
+    vs = [torch.randn_like(k) for k in ks]
+    qb = queries(s, 0, 0, batch=B, device=device)
+    slb = torch.tensor(seq_lens, dtype=torch.int32, device=device)
+    outb = torch.empty(B, s.n_q_heads, s.head_dim, dtype=torch.bfloat16, device=device)
+    wsb2 = torch.empty(L.loopvq_bf16_decode_workspace_bytes(B, s.n_q_heads, s.head_dim, max_len) // 4 + 4,
+                       device=device)
+    bcalls = [lambda st, k=k, v=v: L.loopvq_bf16_decode_attn(qb, k, v, slb, outb, wsb2, stream=st)
+              for k, v in zip(ks, vs)]
+    per_b, _ = time_calls(bcalls, reps=20)
+    row["bf16_us_per_call"] = statistics.median(per_b)
+    row["vq_speedup_vs_bf16"] = row["bf16_us_per_call"] / med
+    del ks, vs
+    torch.cuda.empty_cache()
+    return row
+
+
+def decode_rows(device, peak):
+    """The decode batch sweep (batch 1..256 at context 16384, 16 heads,
+    d = 128, 0.5 bit) and the per-call rows of the other configurations,
+    each beside the same-shape bf16-KV kernel."""
+    import torch
+    from synthetic import SHAPES
+
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    sw = SHAPES["sweep"]
+    sweep = []
+    for B in (1, 2, 4, 8, 16, 32, 64, 128, 256):
+        rot = max(1, min(256 // B, -(-4 * l2 // alg_bytes_per_call(sw, [sw.context] * B))))
+        sweep.append(decode_row(sw.with_(batch=B), [sw.context] * B, 1, [0, sw.n_loops - 1], device,
+                                peak, l2, rotate_seqs=rot))
+    rows = {"sweep": sweep}
+    o = SHAPES["ouro14"]
+    rows["ouro14"] = decode_row(o, [o.context] * o.batch, 4, [0, o.n_loops - 1], device, peak, l2)
+    dp = SHAPES["deep025"]
+    rows["deep025"] = decode_row(dp.with_(n_layers=1), [dp.context] * dp.batch, 1,
+                                 [0, dp.n_loops - 1], device, peak, l2)
+    return rows
 
 
 def encode_prefill(device, reps=3):
@@ -505,6 +678,16 @@ def kmeans_step(device, reps=3):
 # main
 # --------------------------------------------------------------------------
 
+def workload_config(shape, world):
+    """The `config` dict of a line: the same for both arms."""
+    return {"workload": shape.name, "layers": shape.n_layers, "kv_heads": shape.n_kv_heads,
+            "head_dim": shape.head_dim, "loops": shape.n_loops, "g": shape.loop_group,
+            "c": shape.chan_group, "bits_per_element": 8 / shape.D, "batch": shape.batch,
+            "context": shape.context, "prefix": shape.prefix, "recent": shape.recent,
+            "global_batch": shape.batch * world, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2: 277 MB per call, layers rotate"}
+
+
 def main():
     args = parse_args()
     if args.warmup < 3:
@@ -530,9 +713,7 @@ def main():
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": v * shape.n_loops / 1e3, "higher_is_better": False,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": shape.name, "batch": shape.batch, "context": shape.context,
-                           "layers": shape.n_layers, "kv_heads": shape.n_kv_heads,
-                           "head_dim": shape.head_dim, "bits_per_element": 8 / shape.D},
+                "config": workload_config(shape, world),
                 "cpu_baseline": rec,
                 "e2e": {"value": v, "unit": "µs/loop-step", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -550,11 +731,8 @@ def main():
     torch.cuda.synchronize()
     barrier(world)
 
+    # timed region: K whole steps, one pair of events, nothing else on the stream
     K = args.steps
-    n_calls = K * shape.n_loops * shape.n_layers
-    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n_calls)]
-    call_events = list(events)
     ev_start, ev_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clk = ClockSampler(local if world > 1 else 0)
     clk.start()
@@ -563,20 +741,29 @@ def main():
     barrier(world)
     torch.cuda.synchronize()
     ev_start.record(st)
-    pending = list(reversed(events))
     for _ in range(K):
-        wl.step(st, events=pending)
+        wl.step(st)
     ev_end.record(st)
     torch.cuda.synchronize()
     barrier(world)
     clocks = clk.stop()
     elapsed_ms = ev_start.elapsed_time(ev_end)
     elapsed_ms = max_over_ranks(elapsed_ms, world)
-    call_us = [a.elapsed_time(b) * 1e3 for a, b in call_events]
-    avg_call_us = sum(call_us) / len(call_us)
-
     loop_steps = K * shape.n_loops * world
     value, ms_per_step = whole_job_value(elapsed_ms, K, shape.n_loops, world)
+
+    # per-call device times of the decode call (a separate pass, events around
+    # every call): the roofline's launch duration
+    n_calls = max(1, min(K, 3)) * shape.n_loops * shape.n_layers
+    call_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(n_calls)]
+    pending = list(reversed(call_events))
+    torch.cuda.synchronize()
+    for _ in range(max(1, min(K, 3))):
+        wl.step(st, events=pending)
+    torch.cuda.synchronize()
+    call_us = [a.elapsed_time(b) * 1e3 for a, b in call_events]
+    avg_call_us = sum(call_us) / len(call_us)
 
     # end to end through the public API with host buffers: per step the
     # queries, the new token's K/V rows and the evicted token come from
@@ -626,22 +813,16 @@ def main():
                     "sub_bit_vq_b200/csrc/decode.cu", "vq_decode_long32k"),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)" if
                 peak_src == "measured" else "fallback 6650 GB/s",
-                "kernel": "vq_stream_kernel + vq_finish_kernel (per-call events)",
+                "kernel": "vq_pair_kernel + vq_stream_kernel (one decode call, per-call events)",
                 "algorithmic_bytes_per_launch": alg, "avg_launch_us": avg_call_us,
                 "launch_us_p10_median_p90": call_percentiles(call_us),
+                "calls_timed": len(call_us),
                 "frac_of_8tbs": achieved / 8000.0}
 
     line = {"metric": METRIC, "value": value, "unit": "µs/loop-step", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
-            "data": "synthetic",
-            "config": {"workload": shape.name, "layers": shape.n_layers,
-                       "kv_heads": shape.n_kv_heads, "head_dim": shape.head_dim,
-                       "loops": shape.n_loops, "g": shape.loop_group, "c": shape.chan_group,
-                       "bits_per_element": 8 / shape.D, "batch": shape.batch,
-                       "context": shape.context, "prefix": shape.prefix, "recent": shape.recent,
-                       "global_batch": shape.batch * world, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2: 277 MB per call, layers rotate"},
+            "data": "synthetic", "config": workload_config(shape, world),
             "e2e": {"value": e2e_val, "unit": "µs/loop-step", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": wl.launches_per_step() * K,
@@ -654,6 +835,7 @@ def main():
         torch.cuda.empty_cache()
         line["bf16_kv"] = bf16_comparison(shape, dev)
         line["bf16_kv"]["vq_speedup_per_call"] = line["bf16_kv"]["us_per_call"] / avg_call_us
+        line["decode_rows"] = decode_rows(dev, peak)
         line["encode_prefill"] = encode_prefill(dev)
         line["kmeans_step"] = kmeans_step(dev)
     if world > 1:

@@ -230,8 +230,9 @@ loopvq_status loopvq_kmeans_step(const loopvq_config* cfg, int layer, int loop_g
  * Bytes of scratch that loopvq_decode_attn needs for `batch` sequences of
  * at most `max_seq_len` tokens: a 256-byte status area (below), then
  * (batch*Hq + 256) segment records of 4 + head_dim float32 (a segment's
- * softmax maximum and sum and its unnormalised output), then batch*Hq key
- * lookup tables of 256 x J float32. Host only, pure.
+ * softmax maximum and sum and its unnormalised output), batch*Hq window
+ * partials of the same size, batch*Hq key lookup tables of 256 x J float32
+ * and batch*Hq 32-bit record counters. Host only, pure.
  */
 size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int max_seq_len);
 

@@ -168,12 +168,9 @@ loopvq_status loopvq_cache_layout(const loopvq_config* cfg, loopvq_layout* out) 
 size_t loopvq_decode_workspace_bytes(const loopvq_config* cfg, int batch, int max_seq_len) {
   Geometry g;
   if (loopvq::make_geometry(cfg, &g) != LOOPVQ_OK || batch <= 0 || max_seq_len < 0) return 0;
-  // the status word; one record (m, l, two spare floats, unnormalised output
-  // o[d]) per (pair, streaming CTA) segment: record slots pair + cta never
-  // collide, so pairs + CTAs slots suffice; one key lookup table per pair
-  const size_t slots = static_cast<size_t>(batch) * g.Hq + loopvq::kMaxStreamCtas;
-  return loopvq::kStatusBytes + slots * (4 + static_cast<size_t>(g.d)) * sizeof(float) +
-         loopvq::decode_lut_bytes(batch * g.Hq, g.J);
+  // record slots pair + cta of the (pair, streaming CTA) segments never
+  // collide, so pairs + CTAs slots suffice
+  return loopvq::decode_workspace_bytes(batch * g.Hq, g.J, g.d);
 }
 
 loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_idx, int kv,

@@ -1,9 +1,11 @@
 // Fused LoopVQ decode attention over the packed index cache (sm_100a).
 //
-// Three kernels per call, each a programmatic dependent of the one before.
+// Two kernels per call, the second a programmatic dependent of the first.
 //
-// vq_lut_kernel: one CTA per (sequence, query head) pair with quantised
-// tokens builds the pair's key lookup table
+// vq_pair_kernel: per (sequence, query head) pair, one CTA scores the bf16
+// window tokens (prefix + recent) into a window partial (and, for a pair
+// without quantised tokens, writes the result), and J/4 CTAs build the
+// pair's key lookup table
 //     LUT[e][j] = s*log2(e) * q_j . C_K[j][e][tau]
 // (E x J floats) into the workspace.
 //
@@ -36,10 +38,9 @@
 //      of group j), is contracted with the value codebook slice,
 //      o_j = sum_e W[e][j] C_V[j][e][tau], and the segment record
 //      (m, l = sum_e W[e][j], o[d]) goes to slot (pair + cta).
-//
-// vq_finish_kernel: one CTA per pair scores the bf16 window tokens (prefix +
-// recent), merges them with the pair's segment records (log-sum-exp
-// weights) and writes out and lse.
+//   4. The CTA counts its record on the pair's counter; the CTA that writes
+//      the pair's last record merges the window partial with every record
+//      (log-sum-exp weights) and writes out and lse. No CTA waits on another.
 //
 // The hot loops address shared memory by absolute shared-window address: a
 // byte permute puts an index byte into byte 1 of (lane * 4), and the window
@@ -67,8 +68,7 @@ constexpr int kPrefetchPages = 4;         // pages a warp asks L2 to fetch ahead
 constexpr int kFixMax = 30;               // largest fixed-point exponent: w = rn(2^(x - m) * 2^S)
 constexpr float kMassHigh = 2147483648.0f;  // 2^31: lower S before a segment's total passes this
 constexpr int kMassLandLog2 = 29;         // after lowering S the total sits below 2^29
-constexpr int kFinishThreads = 256;
-constexpr int kLutThreads = 256;          // one thread per centroid
+constexpr int kPairThreads = 256;         // window partial: 8 warps; lookup table: one thread per centroid
 constexpr int kWinChunk = 9;              // window tokens per warp per round of loads (72 = 8 warps x 9)
 constexpr int kSegmentUnits = 16;         // work units (pages) charged for a segment's setup
 constexpr int kCols = 64;                 // columns of the shared LUT and histogram
@@ -77,6 +77,7 @@ constexpr int kCols = 64;                 // columns of the shared LUT and histo
 // starts at kSBase (the reserved shared memory of a block on sm_100).
 constexpr uint32_t kSBase = 0x400u;
 constexpr uint32_t kStatOff = 0;          // [2][kNW][2] per-warp chunk maximum and weight sum
+constexpr uint32_t kFlagOff = 0x200u;     // int: last-writer flag
 constexpr uint32_t kSmallBytes = 0x400u;
 constexpr uint32_t kLutAbs = kSBase + kSmallBytes;        // [E][64] floats, 256-byte rows
 constexpr uint32_t kHistAbs = kLutAbs + kE * kCols * 4;   // [E][64] 32-bit words, 256-byte rows
@@ -99,6 +100,8 @@ struct DecodeParams {
   const uint16_t* win_v;
   float* records;                   // [pairs + n_cta][4 + d]: m, l, -, -, o[d]
   float* luts;                      // [pairs][E][J] key lookup tables
+  float* wrecs;                     // [pairs][4 + d]: the bf16 window partial of each pair
+  unsigned* counts;                 // [pairs] segment records written so far (zeroed by the pair kernel)
   int* status;                      // status word (bit flags), never cleared by the kernels
   void* out;
   float* lse;
@@ -375,41 +378,117 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
 
 
 
-// One CTA per pair with quantised tokens: the pair's key lookup table
+// Merges a pair's window partial with its segment records (slots pair + c
+// for the CTAs c in [c_first, c_last] whose unit range is not empty: CTA c
+// of n_cta owns units [U*c/n_cta, U*(c+1)/n_cta)) and writes out and lse.
+// Every thread of the CTA (NT threads) calls it; sh holds 4 + 256 floats.
+// m in log2 units; a record with m = -inf is empty, a NaN m poisons the
+// result.
+template <int D, int NT>
+__device__ void merge_pair(const DecodeParams& p, int pair, int c_first, int c_last, long long U,
+                           float* sh) {
+  constexpr int RS = 4 + D;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const float* wr = p.wrecs + static_cast<size_t>(pair) * RS;
+  const bool every = U >= p.n_cta;                     // then no CTA's range is empty
+  auto written = [&](int c) { return every || U * c / p.n_cta < U * (c + 1) / p.n_cta; };
+  if (tid < 32) {
+    const float m_win = __ldcg(wr);
+    float M = m_win;
+    for (int c = c_first + lane; c <= c_last; c += 32)
+      if (written(c)) M = fmaxf(M, __ldcg(p.records + static_cast<size_t>(pair + c) * RS));
+    M = warp_max(M);
+    float L = 0.f;
+    for (int c = c_first + lane; c <= c_last; c += 32) {
+      float f = 0.f;
+      if (written(c)) {
+        const float* rec = p.records + static_cast<size_t>(pair + c) * RS;
+        const float m = __ldcg(rec);
+        if (m != -INFINITY) {
+          f = fast_exp2(m - M);
+          L += __ldcg(rec + 1) * f;
+        }
+      }
+      sh[4 + c - c_first] = f;
+    }
+    L = warp_sum(L);
+    if (lane == 0) {
+      const float f_win = (m_win == -INFINITY) ? 0.f : fast_exp2(m_win - M);
+      sh[0] = M;
+      sh[1] = L + f_win * __ldcg(wr + 1);
+      sh[2] = f_win;
+    }
+  }
+  __syncthreads();
+  const float M = sh[0], L = sh[1], f_win = sh[2];
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  for (int ch = tid; ch < D; ch += NT) {
+    float o = (f_win != 0.f) ? f_win * __ldcg(wr + 4 + ch) : 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+      const float f = sh[4 + c - c_first];
+      if (f != 0.f) o = fmaf(f, __ldcg(p.records + static_cast<size_t>(pair + c) * RS + 4 + ch), o);
+    }
+    o *= inv;
+    if (p.out_dtype == LOOPVQ_DTYPE_F32)
+      static_cast<float*>(p.out)[static_cast<size_t>(pair) * D + ch] = o;
+    else
+      static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(pair) * D + ch] = __float2bfloat16_rn(o);
+  }
+  if (tid == 0 && p.lse != nullptr)
+    p.lse[pair] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+}
+
+// The per-pair work that needs no index stream, before the streaming
+// kernel: CTA (pair, 0) scores the pair's bf16 window tokens (prefix +
+// recent) and writes the window partial (m, l, -, -, o[d]) to wrecs[pair];
+// CTA (pair, 1 + g) writes groups 4g .. 4g+3 of the pair's key lookup table
 // LUT[e][j] = s*log2(e) * sum_ch q[j*C + ch] * C_K[j][e][tau][ch] into
-// luts[pair][e][j]. Thread e owns centroid e; its loads of C_K[j][e][.] are
-// consecutive across the warp.
+// luts[pair][e][j] (thread e owns centroid e; its loads of C_K[j][e][.] are
+// consecutive across the warp).
 template <int J, int C>
-__global__ void __launch_bounds__(kLutThreads) vq_lut_kernel(const DecodeParams p) {
-  constexpr int d = J * C;
-  static_assert(kLutThreads == kE, "one thread per centroid");
-  __shared__ float qs[d];
-  const int pair = blockIdx.x;
+__global__ void __launch_bounds__(kPairThreads) vq_pair_kernel(const DecodeParams p) {
+  constexpr int D = J * C;
+  constexpr int NW = kPairThreads / 32;
+  constexpr int RS = 4 + D;
+  static_assert(kPairThreads == kE, "one thread per centroid");
+  __shared__ float wst[2 * NW];
+  __shared__ float wpart[NW * D > 8 ? NW * D : 8];
+  __shared__ float wres[D + 2];
+  const int pair = blockIdx.x, part = blockIdx.y;
   const int b = pair / p.Hq, hq = pair % p.Hq, hkv = hq / p.ratio;
   // the streaming kernel may start now; it waits for this grid before it
   // reads a table
   asm volatile("griddepcontrol.launch_dependents;");
-  if (seq_pages(p, b) == 0) return;                    // CTA-uniform: no quantised tokens
-  const int e = threadIdx.x;
-  for (int i = e; i < d; i += kLutThreads)
-    qs[i] = bf16_bits_to_float(p.q[static_cast<size_t>(pair) * d + i]) * p.scale_log2;
-  __syncthreads();
-  const float* cbk = p.cb_k + hkv * p.cb_stride_head;  // [J][E][C]
-  float* out = p.luts + (static_cast<size_t>(pair) * kE + e) * J;
-#pragma unroll 1
-  for (int j0 = 0; j0 < J; j0 += 4) {
-    float v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float cw[C];
-      load_cw<C>(cbk + (static_cast<size_t>(j0 + k) * kE + e) * C, cw);
-      float acc = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < C; ++ch) acc = fmaf(qs[(j0 + k) * C + ch], cw[ch], acc);
-      v[k] = acc;
+  const int tid = threadIdx.x;
+  if (part == 0) {
+    const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
+    window_partial<D, NW>(p, b, hkv, p.q + static_cast<size_t>(pair) * D, min(N, p.W), wst, wpart, wres);
+    float* wr = p.wrecs + static_cast<size_t>(pair) * RS;
+    for (int i = tid; i < D + 2; i += kPairThreads) wr[i < 2 ? i : i + 2] = wres[i];
+    if (tid == 0) p.counts[pair] = 0u;
+    if (seq_pages(p, b) == 0) {                        // window tokens only: the result is final here
+      __syncthreads();
+      merge_pair<D, kPairThreads>(p, pair, 0, -1, 1, wpart);
     }
-    *reinterpret_cast<float4*>(out + j0) = make_float4(v[0], v[1], v[2], v[3]);
+    return;
   }
+  if (seq_pages(p, b) == 0) return;                    // CTA-uniform: no quantised tokens
+  const int j0 = (part - 1) * 4, e = tid;
+  const float* cbk = p.cb_k + hkv * p.cb_stride_head;  // [J][E][C]
+  const uint16_t* qp = p.q + static_cast<size_t>(pair) * D + j0 * C;
+  float cw[4][C];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) load_cw<C>(cbk + (static_cast<size_t>(j0 + k) * kE + e) * C, cw[k]);
+  float v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float acc = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < C; ++ch) acc = fmaf(bf16_bits_to_float(qp[k * C + ch]) * p.scale_log2, cw[k][ch], acc);
+    v[k] = acc;
+  }
+  *reinterpret_cast<float4*>(p.luts + (static_cast<size_t>(pair) * kE + e) * J + j0) =
+      make_float4(v[0], v[1], v[2], v[3]);
 }
 
 template <int J, int C>
@@ -444,9 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   // the finish kernel may start its window work as SMs free up; it waits for
   // this grid before it reads the records
   asm volatile("griddepcontrol.launch_dependents;");
-  if (u_lo >= u_hi) return;                            // CTA-uniform
+  if (u_lo >= u_hi) {                                  // CTA-uniform
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // this grid completes after the one before
+    return;
+  }
   int b;
-  long long pre;
+  long long pre;                                       // units of one head of the sequences before b
   find_unit(p, u_lo, lane, &b, &pre);
   int units_b = pair_units(seq_pages(p, b));
   const long long off = u_lo - static_cast<long long>(p.Hq) * pre;
@@ -455,6 +537,14 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
   long long u = u_lo;
   if (bad_base && tid == 0 && p.status != nullptr) atomicOr(p.status, kStatusSharedBase);
   bool tables_ready = false;
+  // the pair kernel's tables, window partials and zeroed counters
+  auto ensure_ready = [&]() {
+    if (!tables_ready) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      tables_ready = true;
+    }
+  };
+  int* s_last = reinterpret_cast<int*>(smem_u8 + kFlagOff);   // this CTA wrote a pair's last record
 
   while (u < u_hi && b < p.B) {
     const int seg_units = static_cast<int>(min(static_cast<long long>(units_b - pu_start), u_hi - u));
@@ -552,19 +642,27 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       issue_keys(0);
 #pragma unroll
       for (int q = 0; q < KB; ++q) issue_key(0, q);
-      if (!tables_ready) {                             // the LUT kernel's tables are complete
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        tables_ready = true;
-      }
+      ensure_ready();
       {
+        constexpr int NF = kE * J / 4;                 // float4s of the table
+        constexpr int PER = (NF + kThreads - 1) / kThreads;
         const float4* src = reinterpret_cast<const float4*>(p.luts + static_cast<size_t>(pair) * kE * J);
-        for (int f = tid; f < kE * J / 4; f += kThreads) {
-          const float4 v = __ldcg(src + f);
-          const int e = f / (J / 4), c0 = (f - e * (J / 4)) * 4;
-          for (int c = c0; c + 4 <= kCols; c += J) *reinterpret_cast<float4*>(lut + e * kCols + c) = v;
-        }
+        float4 v[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k)
+          if (tid + k * kThreads < NF) v[k] = __ldcg(src + tid + k * kThreads);
+#pragma unroll
         for (int i = tid * 4; i < kE * kCols; i += kThreads * 4)
           *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int f = tid + k * kThreads;
+          if (f < NF) {
+            const int e = f / (J / 4), c0 = (f - e * (J / 4)) * 4;
+#pragma unroll
+            for (int c = c0; c + 4 <= kCols; c += J) *reinterpret_cast<float4*>(lut + e * kCols + c) = v[k];
+          }
+        }
       }
       __syncthreads();                                 // LUT and histogram ready
 
@@ -721,109 +819,40 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       }
     }
 
+    // ---- publish the record; the pair's last writer merges ------------------
+    {
+      // the CTAs whose unit ranges meet the pair's units [u0, u0 + units_b)
+      const long long u0 = pre * p.Hq + static_cast<long long>(hq) * units_b;
+      const int c_first = static_cast<int>(((u0 + 1) * p.n_cta - 1) / U);
+      const int c_last = static_cast<int>(((u0 + units_b) * p.n_cta - 1) / U);
+      ensure_ready();                                  // the counter was zeroed by the pair kernel
+      __threadfence();                                 // this thread's record writes, device-wide
+      __syncthreads();
+      if (tid == 0) {
+        int n = c_last - c_first + 1;                  // writers: the CTAs of the range with units
+        if (U < p.n_cta)
+          for (int c = c_first; c <= c_last; ++c) n -= (U * c / p.n_cta < U * (c + 1) / p.n_cta) ? 0 : 1;
+        *s_last = atomicAdd(p.counts + pair, 1u) == static_cast<unsigned>(n - 1);
+      }
+      __syncthreads();
+      if (*s_last) {                                   // CTA-uniform: every record of the pair is written
+        __threadfence();
+        merge_pair<d, kThreads>(p, pair, c_first, c_last, U, lut);
+      }
+    }
+
     u += seg_units;
     pu_start = 0;
     if (++hq == p.Hq) {
       hq = 0;
       do {
+        pre += units_b;
         ++b;
       } while (b < p.B && u < u_hi && (units_b = pair_units(seq_pages(p, b))) == 0);
     }
   }
-  if (!tables_ready) asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-// One CTA per (sequence, query head): the bf16 window partial and the merge
-// of the pair's segment records (log-sum-exp weights); writes out and lse.
-template <int J, int C>
-__global__ void __launch_bounds__(kFinishThreads) vq_finish_kernel(const DecodeParams p) {
-  constexpr int D = J * C;
-  constexpr int NW = kFinishThreads / 32;
-  constexpr int RS = 4 + D;                            // record floats
-  __shared__ float wst[2 * NW];
-  __shared__ float wpart[NW * D];
-  __shared__ float wres[D + 2];
-  __shared__ float fc[kMaxStreamCtas];
-  __shared__ float sstat[4];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int pair = blockIdx.x;
-  const int b = pair / p.Hq, hq = pair % p.Hq, hkv = hq / p.ratio;
-  const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
-  const int pages_b = seq_pages(p, b);                 // CTA-uniform
-  window_partial<D, NW>(p, b, hkv, p.q + static_cast<size_t>(pair) * D, min(N, p.W), wst, wpart, wres);
-
-  // the pair's segment records: slots pair + c for the CTAs c that own its units
-  int c_first = 0, c_last = -1;
-  long long U = 1;
-  if (pages_b > 0) {
-    int bb;
-    long long pre;
-    U = find_unit(p, -1, lane, &bb, &pre);
-    long long before = 0;                              // units of one head of sequences < b
-    for (int b0 = 0; b0 < b; b0 += 32) {
-      const int bi = b0 + lane;
-      long long v = (bi < b) ? static_cast<long long>(pair_units(seq_pages(p, bi))) : 0;
-      v = warp_incl_scan(v, lane);
-      before += __shfl_sync(0xffffffffu, v, 31);
-    }
-    const int units_b = pair_units(pages_b);
-    const long long u0 = before * p.Hq + static_cast<long long>(hq) * units_b;
-    c_first = static_cast<int>(((u0 + 1) * p.n_cta - 1) / U);
-    c_last = static_cast<int>(((u0 + units_b) * p.n_cta - 1) / U);
-  }
-  // everything above reads only inputs; the segment records need the
-  // streaming kernel to be complete
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // a CTA whose unit range is empty wrote no record
-  auto rec_of = [&](int c) -> const float* {
-    return (U * c / p.n_cta < U * (c + 1) / p.n_cta)
-               ? p.records + static_cast<size_t>(pair + c) * RS : nullptr;
-  };
-  if (warp == 0) {
-    float M = wres[0];
-    for (int c = c_first + lane; c <= c_last; c += 32) {
-      const float* rec = rec_of(c);
-      if (rec != nullptr) M = fmaxf(M, __ldcg(rec));
-    }
-    M = warp_max(M);
-    float L = 0.f;
-    for (int c = c_first + lane; c <= c_last; c += 32) {
-      const float* rec = rec_of(c);
-      float f = 0.f;
-      if (rec != nullptr) {
-        const float m = __ldcg(rec);
-        if (m != -INFINITY) {
-          f = fast_exp2(m - M);                          // NaN m (a timed-out turn) poisons M and L
-          L += __ldcg(rec + 1) * f;
-        }
-      }
-      fc[c - c_first] = f;
-    }
-    L = warp_sum(L);
-    if (lane == 0) {
-      const float f_win = (wres[0] == -INFINITY) ? 0.f : fast_exp2(wres[0] - M);
-      sstat[0] = M;
-      sstat[1] = L + f_win * wres[1];
-      sstat[2] = f_win;
-    }
-  }
-  __syncthreads();
-  const float M = sstat[0], L = sstat[1], f_win = sstat[2];
-  const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  for (int ch = tid; ch < D; ch += kFinishThreads) {
-    float o = (f_win != 0.f) ? f_win * wres[2 + ch] : 0.f;
-    for (int c = c_first; c <= c_last; ++c) {
-      const float f = fc[c - c_first];
-      if (f != 0.f) o = fmaf(f, __ldcg(p.records + static_cast<size_t>(pair + c) * RS + 4 + ch), o);
-    }
-    o *= inv;
-    if (p.out_dtype == LOOPVQ_DTYPE_F32)
-      static_cast<float*>(p.out)[static_cast<size_t>(pair) * D + ch] = o;
-    else
-      static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(pair) * D + ch] = __float2bfloat16_rn(o);
-  }
-  if (tid == 0 && p.lse != nullptr)
-    p.lse[pair] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+  // every CTA waits once, so that this grid completes after the pair kernel
+  ensure_ready();
 }
 
 template <typename K>
@@ -874,23 +903,27 @@ template <int J, int C>
 loopvq_status launch_vq(const DecodeParams& p, cudaStream_t st, bool run_stream) {
   static_assert(kDynBytes <= 227 * 1024, "streaming kernel shared memory above 227 KB");
   const unsigned pairs = static_cast<unsigned>(p.B * p.Hq);
+  // window partials, and the key tables when anything streams
+  vq_pair_kernel<J, C><<<dim3(pairs, run_stream ? 1 + J / 4 : 1), kPairThreads, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return LOOPVQ_ERR_CUDA;
   if (run_stream) {
     static std::atomic<uint64_t> configured{0};
     const loopvq_status s = set_smem(vq_stream_kernel<J, C>, kDynBytes, configured);
     if (s != LOOPVQ_OK) return s;
-    vq_lut_kernel<J, C><<<pairs, kLutThreads, 0, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return LOOPVQ_ERR_CUDA;
-    const loopvq_status s2 =
-        launch_dependent(vq_stream_kernel<J, C>, static_cast<unsigned>(p.n_cta), kThreads, kDynBytes, st, p);
-    if (s2 != LOOPVQ_OK) return s2;
+    return launch_dependent(vq_stream_kernel<J, C>, static_cast<unsigned>(p.n_cta), kThreads, kDynBytes, st,
+                            p);
   }
-  return launch_dependent(vq_finish_kernel<J, C>, pairs, kFinishThreads, 0, st, p);
+  return LOOPVQ_OK;
 }
 
 }  // namespace
 
-size_t decode_lut_bytes(int pairs, int J) {
-  return static_cast<size_t>(pairs) * kE * J * sizeof(float);
+size_t decode_workspace_bytes(int pairs, int J, int d) {
+  const size_t rec = (4 + static_cast<size_t>(d)) * sizeof(float);
+  return kStatusBytes + (static_cast<size_t>(pairs) + kMaxStreamCtas) * rec +   // segment records
+         static_cast<size_t>(pairs) * rec +                                     // window partials
+         static_cast<size_t>(pairs) * kE * J * sizeof(float) +                  // key lookup tables
+         (static_cast<size_t>(pairs) * sizeof(unsigned) + 15) / 16 * 16;        // record counters
 }
 
 loopvq_status launch_decode(const DecodeArgs& a) {
@@ -917,9 +950,11 @@ loopvq_status launch_decode(const DecodeArgs& a) {
   char* ws = static_cast<char*>(a.workspace);
   const size_t pairs = static_cast<size_t>(a.batch) * g.Hq;
   p.status = reinterpret_cast<int*>(ws);
+  const size_t rec = (4 + static_cast<size_t>(g.d)) * sizeof(float);
   p.records = reinterpret_cast<float*>(ws + kStatusBytes);
-  p.luts = reinterpret_cast<float*>(ws + kStatusBytes +
-                                    (pairs + kMaxStreamCtas) * (4 + static_cast<size_t>(g.d)) * sizeof(float));
+  p.wrecs = reinterpret_cast<float*>(ws + kStatusBytes + (pairs + kMaxStreamCtas) * rec);
+  p.luts = reinterpret_cast<float*>(ws + kStatusBytes + (2 * pairs + kMaxStreamCtas) * rec);
+  p.counts = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(p.luts) + pairs * kE * g.J * sizeof(float));
   p.out = a.out;
   p.lse = a.lse;
   p.B = a.batch;

@@ -29,12 +29,14 @@ int max_decode_splits(int pairs, int pages);
 constexpr int kMaxStreamCtas = 256;
 
 // Bytes at the start of the decode workspace that hold the status word (an
-// int32 of flag bits); the segment records follow, then one key lookup table
-// of E x J floats per (sequence, query head) pair.
+// int32 of flag bits).
 constexpr size_t kStatusBytes = 256;
 
-// Bytes of the key lookup tables of `pairs` pairs with J channel groups.
-size_t decode_lut_bytes(int pairs, int J);
+// Decode workspace of `pairs` (sequence, query head) pairs: the status word,
+// (pairs + kMaxStreamCtas) segment records and `pairs` window partials of
+// 4 + d floats, one key lookup table of E x J floats per pair, and one
+// 32-bit record counter per pair.
+size_t decode_workspace_bytes(int pairs, int J, int d);
 
 // Number of multiprocessors of the current device (cached per device).
 // Returns 0 and sets *err when the runtime fails.

@@ -172,12 +172,14 @@ def test_kmeans_step_rejects_before_launch():
 def test_workspace_bytes_formula():
     cfg = _cfg()
     # a 256-byte status area, then one record (m, l, 2 spare, o[d]) of float32
-    # per (pair, streaming CTA) slot: pairs + 256 slots, then one key lookup
-    # table of 256 x J float32 per pair
+    # per (pair, streaming CTA) slot: pairs + 256 slots, one window partial of
+    # the same size per pair, one key lookup table of 256 x J float32 per
+    # pair and one 32-bit record counter per pair (rounded up to 16 bytes)
     n = L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64)
     rec = 4 * (4 + cfg.head_dim)
     pairs, J = 2 * cfg.n_q_heads, cfg.head_dim // cfg.chan_group
-    assert n == 256 + rec * (pairs + 256) + pairs * 256 * J * 4
+    counters = -(-pairs * 4 // 16) * 16
+    assert n == 256 + rec * (pairs + 256) + rec * pairs + pairs * 256 * J * 4 + counters
     # more sequences need more records
     assert L.loopvq_decode_workspace_bytes(cfg, 4, 72 + 5 * 64) > n
     assert L.loopvq_decode_workspace_bytes(cfg, 0, 10) == 0
