@@ -5,6 +5,8 @@ loads it and marshals arguments. Importing it without the built library
 raises ``ImportError``: there is no CPU fallback.
 """
 from .binding import (  # noqa: F401
+    LOOPVQ_DECODE_STATUS_BAD_PAGE,
+    LOOPVQ_DECODE_STATUS_SHARED_BASE,
     LOOPVQ_DTYPE_BF16,
     LOOPVQ_DTYPE_F32,
     LoopVQConfig,

@@ -25,6 +25,8 @@ LOOPVQ_ERR_WORKSPACE = 3
 LOOPVQ_ERR_CUDA = 4
 LOOPVQ_DTYPE_BF16 = 0
 LOOPVQ_DTYPE_F32 = 1
+LOOPVQ_DECODE_STATUS_BAD_PAGE = 1
+LOOPVQ_DECODE_STATUS_SHARED_BASE = 2
 
 
 class LoopVQError(RuntimeError):

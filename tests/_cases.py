@@ -16,6 +16,8 @@ import sub_bit_vq_b200 as L
 from oracle import loopvq_oracle as O
 from synthetic import Shape, block_tables, codebooks_for_layer, queries, window_kv
 
+from _guard import Guarded, status_word, workspace
+
 TOL_F32_REL = 1e-4      # fp32 output: per-row max|o - ref| / max|ref|
 TOL_BF16_ABS = 2e-2     # bf16 output: max abs, floored at one bf16 ulp of ref
 TOL_LSE = 1e-4
@@ -110,14 +112,17 @@ class DecodeCase:
         q = self.q.to(dev)
         wk, wv = self.win_k.to(dev), self.win_v.to(dev)
         s = self.shape
-        out = torch.full((self.B, s.n_q_heads, s.head_dim), float("nan"), dtype=out_dtype, device=dev)
-        lse = torch.full((self.B, s.n_q_heads), float("nan"), dtype=torch.float32, device=dev)
-        nbytes = L.loopvq_decode_workspace_bytes(cfg, self.B, self.max_seq_len)
-        ws = torch.full((max(nbytes // 4, 1),), float("nan"), dtype=torch.float32, device=dev)
-        L.loopvq_decode_attn(cfg, self.layer, self.t, q, pool, cb, bt, sl, wk, wv, out, ws,
-                             self.max_seq_len, lse=lse, sm_scale=self.sm_scale)
+        out = Guarded((self.B, s.n_q_heads, s.head_dim), out_dtype, fill=float("nan"), device=dev)
+        lse = Guarded((self.B, s.n_q_heads), torch.float32, fill=float("nan"), device=dev)
+        ws = workspace(L.loopvq_decode_workspace_bytes(cfg, self.B, self.max_seq_len), device=dev)
+        L.loopvq_decode_attn(cfg, self.layer, self.t, q, pool, cb, bt, sl, wk, wv, out.t, ws.t,
+                             self.max_seq_len, lse=lse.t, sm_scale=self.sm_scale)
         torch.cuda.synchronize()
-        return out.float().cpu().numpy(), lse.cpu().numpy()
+        out.check("output")
+        lse.check("lse")
+        ws.check("workspace")
+        assert status_word(ws) == 0, f"decode status {status_word(ws)}"
+        return out.t.float().cpu().numpy(), lse.t.cpu().numpy()
 
 
 def check_decode(case: DecodeCase, out: np.ndarray, lse: np.ndarray, out_dtype, pairs=None):
@@ -219,14 +224,17 @@ class DeviceDecodeCase:
         cb, bt = self.cb.to(dev), self.bt.to(dev)
         sl = torch.tensor(self.seq_lens, dtype=torch.int32, device=dev)
         q, wk, wv = self.q.to(dev), self.win_k.to(dev), self.win_v.to(dev)
-        out = torch.full((self.B, s.n_q_heads, s.head_dim), float("nan"), dtype=out_dtype, device=dev)
-        lse = torch.full((self.B, s.n_q_heads), float("nan"), dtype=torch.float32, device=dev)
-        nbytes = L.loopvq_decode_workspace_bytes(cfg, self.B, self.max_seq_len)
-        ws = torch.full((max(nbytes // 4, 1),), float("nan"), dtype=torch.float32, device=dev)
-        L.loopvq_decode_attn(cfg, self.layer, self.t, q, self.pool, cb, bt, sl, wk, wv, out, ws,
-                             self.max_seq_len, lse=lse, sm_scale=self.sm_scale)
+        out = Guarded((self.B, s.n_q_heads, s.head_dim), out_dtype, fill=float("nan"), device=dev)
+        lse = Guarded((self.B, s.n_q_heads), torch.float32, fill=float("nan"), device=dev)
+        ws = workspace(L.loopvq_decode_workspace_bytes(cfg, self.B, self.max_seq_len), device=dev)
+        L.loopvq_decode_attn(cfg, self.layer, self.t, q, self.pool, cb, bt, sl, wk, wv, out.t, ws.t,
+                             self.max_seq_len, lse=lse.t, sm_scale=self.sm_scale)
         torch.cuda.synchronize()
-        return out.float().cpu().numpy(), lse.cpu().numpy()
+        out.check("output")
+        lse.check("lse")
+        ws.check("workspace")
+        assert status_word(ws) == 0, f"decode status {status_word(ws)}"
+        return out.t.float().cpu().numpy(), lse.t.cpu().numpy()
 
 
 def sample_pairs(B: int, Hq: int, n: int, seed: int, whole=()):

@@ -210,3 +210,11 @@ def test_static_scratch_size_matches_the_header():
     assert m, "LOOPVQ_STATIC_SCRATCH_BYTES not found in include/loopvq.h"
     assert int(m.group(1)) << int(m.group(2)) == B.LOOPVQ_STATIC_SCRATCH_BYTES
     assert L.LOOPVQ_STATIC_SCRATCH_BYTES == B.LOOPVQ_STATIC_SCRATCH_BYTES
+
+
+def test_status_bits_match_the_header():
+    text = open(os.path.join(ROOT, "include", "loopvq.h")).read()
+    for name in ("LOOPVQ_DECODE_STATUS_BAD_PAGE", "LOOPVQ_DECODE_STATUS_SHARED_BASE"):
+        m = re.search(name + r"\s*=\s*(\d+)", text)
+        assert m, name
+        assert getattr(B, name) == int(m.group(1)) == getattr(L, name)

@@ -11,6 +11,7 @@ import sub_bit_vq_b200 as L
 from oracle import loopvq_oracle as O
 
 from _cases import TOL_F32_REL, TOL_LSE, TOL_BF16_ABS, bf16_ulp
+from _guard import Guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -24,13 +25,14 @@ def test_bf16_kv_decode(d, dt):
     q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
     k = torch.randn(B, Hkv, S, d, generator=g).to(torch.bfloat16)
     v = torch.randn(B, Hkv, S, d, generator=g).to(torch.bfloat16)
-    out = torch.full((B, Hq, d), float("nan"), dtype=dt, device="cuda")
-    lse = torch.full((B, Hq), float("nan"), device="cuda")
-    ws = torch.empty(L.loopvq_bf16_decode_workspace_bytes(B, Hq, d, S) // 4 + 1, device="cuda")
+    out = Guarded((B, Hq, d), dt, fill=float("nan"))
+    lse = Guarded((B, Hq), torch.float32, fill=float("nan"))
+    ws = Guarded((L.loopvq_bf16_decode_workspace_bytes(B, Hq, d, S) // 4,), torch.float32)
     L.loopvq_bf16_decode_attn(q.cuda(), k.cuda(), v.cuda(),
-                              torch.tensor(seq, dtype=torch.int32, device="cuda"), out, ws, lse=lse)
-    torch.cuda.synchronize()
-    o, ls = out.float().cpu().numpy(), lse.cpu().numpy()
+                              torch.tensor(seq, dtype=torch.int32, device="cuda"), out.t, ws.t, lse=lse.t)
+    for g_, what in ((out, "output"), (lse, "lse"), (ws, "workspace")):
+        g_.check(what)
+    o, ls = out.t.float().cpu().numpy(), lse.t.cpu().numpy()
     scale = 1 / math.sqrt(d)
     for b in range(B):
         for h in range(Hq):

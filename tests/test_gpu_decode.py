@@ -134,3 +134,53 @@ def test_every_dispatched_group_shape(shape):
     case = DecodeCase(shape, [73, 640, 2500], loop_step=2, seed=40)
     out, lse = case.run_gpu(torch.float32)
     check_decode(case, out, lse, torch.float32)
+
+
+def test_out_of_range_page_entries_are_skipped_and_flagged():
+    # Block-table entries outside [0, n_pages) are not read: the kernel skips
+    # those pages, sets LOOPVQ_DECODE_STATUS_BAD_PAGE in the workspace's status
+    # word, and the result is attention over the remaining tokens.
+    import math as _m
+
+    import sub_bit_vq_b200 as L
+    from oracle import loopvq_oracle as O
+
+    from _guard import Guarded, status_word, workspace
+
+    s = RAG128
+    case = DecodeCase(s, [400, 1000], seed=6)
+    good = case.bt.clone()
+    bad = good.clone()
+    bad[1, 2] = case.n_pages + 7                     # past the pool
+    bad[1, 5] = -3                                   # negative
+    dev = "cuda"
+    cfg = case.config()
+    out = Guarded((case.B, s.n_q_heads, s.head_dim), torch.float32, fill=float("nan"))
+    lse = Guarded((case.B, s.n_q_heads), torch.float32, fill=float("nan"))
+    ws = workspace(L.loopvq_decode_workspace_bytes(cfg, case.B, case.max_seq_len))
+    L.loopvq_decode_attn(cfg, 0, case.t, case.q.to(dev), torch.from_numpy(case.pool).to(dev),
+                         case.cb.to(dev), bad.to(dev),
+                         torch.tensor(case.seq_lens, dtype=torch.int32, device=dev),
+                         case.win_k.to(dev), case.win_v.to(dev), out.t, ws.t, case.max_seq_len,
+                         lse=lse.t, sm_scale=case.sm_scale)
+    for g_, what in ((out, "output"), (lse, "lse"), (ws, "workspace")):
+        g_.check(what)
+    assert status_word(ws) & L.LOOPVQ_DECODE_STATUS_BAD_PAGE
+    o, ls = out.t.cpu().numpy(), lse.t.cpu().numpy()
+    # sequence 0 is untouched; sequence 1 lost the tokens of its logical pages 2 and 5
+    for h in range(s.n_q_heads):
+        ref, lref = case.oracle(0, h)
+        assert np.max(np.abs(o[0, h] - ref)) / np.max(np.abs(ref)) <= 1e-4
+        iK, iV = case.indices(1, h)
+        keep = np.ones(iK.shape[0], dtype=bool)
+        for pg in (2, 5):
+            keep[pg * s.page_tokens:(pg + 1) * s.page_tokens] = False
+        nw = O.n_window_tokens(case.seq_lens[1], s.prefix, s.recent)
+        ref, lref = O.decode_attn_ref(case.q[1, h].double().numpy(),
+                                      case.win_k[1, h, :nw].double().numpy(),
+                                      case.win_v[1, h, :nw].double().numpy(), iK[keep], iV[keep],
+                                      case.cb[0, h, 0, 0].double().numpy(),
+                                      case.cb[0, h, 0, 1].double().numpy(), case.tau,
+                                      1.0 / _m.sqrt(s.head_dim))
+        assert np.max(np.abs(o[1, h] - ref)) / np.max(np.abs(ref)) <= 1e-4
+        assert abs(ls[1, h] - lref) <= 1e-4

@@ -13,6 +13,8 @@ from synthetic import SHAPES, Shape, codebooks_for_layer, loop_group_kv, weights
 
 from _cases import check_indices, random_codebooks
 
+from _guard import Guarded
+
 pytestmark = pytest.mark.gpu
 
 W128 = Shape("w128", n_layers=2, n_kv_heads=2, n_q_heads=2, head_dim=128, n_loops=8,
@@ -31,13 +33,13 @@ def _cfg(s: Shape, n_layers: int, n_pages: int) -> L.LoopVQConfig:
 
 def _run(s, n_layers, layer, gamma, kv, x, w, cb, slots, n_pages):
     cfg = _cfg(s, n_layers, n_pages)
-    pool = torch.zeros(n_layers, s.n_kv_heads, s.G, n_pages, 2, s.page_tokens * s.J,
-                       dtype=torch.uint8, device="cuda")
+    pool = Guarded((n_layers, s.n_kv_heads, s.G, n_pages, 2, s.page_tokens * s.J), torch.uint8,
+                   fill=0)
     L.loopvq_encode(cfg, layer, gamma, kv, x.cuda() if x.device.type == "cpu" else x,
                     None if w is None else w.cuda(), cb.cuda(),
-                    torch.as_tensor(slots, dtype=torch.int64).cuda(), pool)
-    torch.cuda.synchronize()
-    return pool.cpu().numpy()
+                    torch.as_tensor(slots, dtype=torch.int64).cuda(), pool.t)
+    pool.check("pool")
+    return pool.t.cpu().numpy()
 
 
 def _gpu_indices(pool, s, layer, gamma, kv, slots):

@@ -15,6 +15,7 @@ from oracle import loopvq_oracle as O
 from synthetic import Shape, loop_group_kv, weights
 
 from _cases import check_indices, random_codebooks
+from _guard import Guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -37,12 +38,11 @@ def _cfg(s: Shape, n_layers: int) -> L.LoopVQConfig:
 def _step(s, n_layers, layer, gamma, kv, x, w, cb_gpu):
     cfg = _cfg(s, n_layers)
     n = x.shape[1]
-    assign = torch.full((L.loopvq_kmeans_assign_bytes(cfg, n),), 255, dtype=torch.uint8,
-                        device="cuda")
+    assign = Guarded((L.loopvq_kmeans_assign_bytes(cfg, n),), torch.uint8, fill=255)
     L.loopvq_kmeans_step(cfg, layer, gamma, kv, x.cuda(), None if w is None else w.cuda(),
-                         cb_gpu, assign)
-    torch.cuda.synchronize()
-    return assign.cpu().numpy().reshape(s.n_kv_heads, s.J, n).transpose(2, 0, 1)   # [n][H][J]
+                         cb_gpu, assign.t)
+    assign.check("assignment")
+    return assign.t.cpu().numpy().reshape(s.n_kv_heads, s.J, n).transpose(2, 0, 1)   # [n][H][J]
 
 
 def _check_step(s, x, w, cb_old, a_gpu, cb_new_gpu):

@@ -20,6 +20,7 @@ from sub_bit_vq_b200 import binding as B
 from synthetic import Shape
 
 from _cases import TOL_F32_REL, TOL_LSE, DecodeCase
+from _guard import Guarded, status_word, workspace
 
 pytestmark = pytest.mark.gpu
 
@@ -42,22 +43,24 @@ def _workspace_reference(case, a):
     """out/lse of the workspace entry point, its scratch filled with NaN."""
     need = L.loopvq_decode_workspace_bytes(a["cfg"], case.B, case.max_seq_len)
     assert 0 < need <= B.LOOPVQ_STATIC_SCRATCH_BYTES
-    ws = torch.full((need // 4 + 1,), float("nan"), device="cuda")
+    ws = workspace(need)
     L.loopvq_decode_attn(a["cfg"], case.layer, case.t, a["q"], a["pool"], a["cb"], a["bt"], a["sl"],
-                         a["wk"], a["wv"], a["out"], ws, case.max_seq_len, lse=a["lse"],
+                         a["wk"], a["wv"], a["out"], ws.t, case.max_seq_len, lse=a["lse"],
                          sm_scale=case.sm_scale)
-    torch.cuda.synchronize()
+    ws.check("workspace")
+    assert status_word(ws) == 0
     return a["out"].cpu().numpy(), a["lse"].cpu().numpy()
 
 
 def _noalloc(case, a):
-    out = torch.full_like(a["out"], float("nan"))
-    lse = torch.full_like(a["lse"], float("nan"))
+    out = Guarded(a["out"].shape, a["out"].dtype, fill=float("nan"))
+    lse = Guarded(a["lse"].shape, a["lse"].dtype, fill=float("nan"))
     B.loopvq_decode_attn_noalloc(a["cfg"], case.layer, case.t, a["q"], a["pool"], a["cb"],
-                                 a["bt"], a["sl"], a["wk"], a["wv"], out, case.max_seq_len,
-                                 lse=lse, sm_scale=case.sm_scale)
-    torch.cuda.synchronize()
-    return out.cpu().numpy(), lse.cpu().numpy()
+                                 a["bt"], a["sl"], a["wk"], a["wv"], out.t, case.max_seq_len,
+                                 lse=lse.t, sm_scale=case.sm_scale)
+    out.check("output")
+    lse.check("lse")
+    return out.t.cpu().numpy(), lse.t.cpu().numpy()
 
 
 def _compare(case, got, ref):
