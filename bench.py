@@ -255,7 +255,7 @@ class Workload:
         self.out = torch.empty(s.n_layers, T, B, Hq, d, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(s.n_layers, T, B, Hq, dtype=torch.float32, device=device)
         ws = L.loopvq_decode_workspace_bytes(self.cfg, B, self.max_seq_len)
-        self.ws = torch.empty(ws // 4 + 4, dtype=torch.float32, device=device)
+        self.ws = torch.zeros(ws // 4 + 4, dtype=torch.float32, device=device)   # zero counters
         # eviction encode inputs: the token leaving the recent window, g loops
         self.evict = torch.empty(s.n_layers, G, 2, g, B, H, d, dtype=torch.bfloat16, device=device)
         for l in range(s.n_layers):
@@ -504,7 +504,7 @@ def decode_row(shape, seq_lens, n_layers, loop_steps, device, peak, l2_bytes, ro
         wv = window_kv(s, l, t, 1, batch=nb, device=device)[r * B:(r + 1) * B].contiguous()
         out = torch.empty(B, s.n_q_heads, s.head_dim, dtype=torch.bfloat16, device=device)
         lse = torch.empty(B, s.n_q_heads, device=device)
-        ws = torch.empty(wsb // 4 + 4, device=device)
+        ws = torch.zeros(wsb // 4 + 4, device=device)
         btr, slr = bt[r * B:(r + 1) * B], sl_all[r * B:(r + 1) * B]
         keep.append((q, wk, wv, out, lse, ws, btr, slr))
 

@@ -393,29 +393,36 @@ __device__ void merge_pair(const DecodeParams& p, int pair, int c_first, int c_l
   const bool every = U >= p.n_cta;                     // then no CTA's range is empty
   auto written = [&](int c) { return every || U * c / p.n_cta < U * (c + 1) / p.n_cta; };
   if (tid < 32) {
-    const float m_win = __ldcg(wr);
+    // (m, l) of the window partial and of up to 32 records per round, loaded together
+    const float m_win = __ldcg(wr), l_win = __ldcg(wr + 1);
     float M = m_win;
-    for (int c = c_first + lane; c <= c_last; c += 32)
-      if (written(c)) M = fmaxf(M, __ldcg(p.records + static_cast<size_t>(pair + c) * RS));
+    float mc[8], lc[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int c = c_first + lane + 32 * r;
+      mc[r] = -INFINITY;
+      lc[r] = 0.f;
+      if (c <= c_last && written(c)) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.records + static_cast<size_t>(pair + c) * RS));
+        mc[r] = ml.x;
+        lc[r] = ml.y;
+      }
+      M = fmaxf(M, mc[r]);
+    }
     M = warp_max(M);
     float L = 0.f;
-    for (int c = c_first + lane; c <= c_last; c += 32) {
-      float f = 0.f;
-      if (written(c)) {
-        const float* rec = p.records + static_cast<size_t>(pair + c) * RS;
-        const float m = __ldcg(rec);
-        if (m != -INFINITY) {
-          f = fast_exp2(m - M);
-          L += __ldcg(rec + 1) * f;
-        }
-      }
-      sh[4 + c - c_first] = f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int c = c_first + lane + 32 * r;
+      const float f = (mc[r] == -INFINITY) ? 0.f : fast_exp2(mc[r] - M);   // a NaN m poisons M and L
+      L += lc[r] * f;
+      if (c <= c_last) sh[4 + c - c_first] = f;
     }
     L = warp_sum(L);
     if (lane == 0) {
       const float f_win = (m_win == -INFINITY) ? 0.f : fast_exp2(m_win - M);
       sh[0] = M;
-      sh[1] = L + f_win * __ldcg(wr + 1);
+      sh[1] = L + f_win * l_win;
       sh[2] = f_win;
     }
   }
@@ -664,8 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           }
         }
       }
-      __syncthreads();                                 // LUT and histogram ready
-
+      __syncthreads();                                 // LUT and histogram ready, staging area free
       // ---- stream -------------------------------------------------------------
       auto key_score = [&](const BlockRegs<J>& r, int nv) -> float {
         if (nv <= 0) return -INFINITY;                 // warp-uniform
@@ -766,6 +772,19 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           rec[1] = 0.f;
         }
       } else {
+        // this warp's groups j = warp + kNW*jw of the value slice, requested
+        // before the histogram is read so that the loads land meanwhile
+        constexpr int JPW = (J + kNW - 1) / kNW;
+        float cv[JPW][kE / 32][C];
+#pragma unroll
+        for (int jw = 0; jw < JPW; ++jw) {
+          const int j = warp + kNW * jw;
+          if (j < J) {
+#pragma unroll
+            for (int i = 0; i < kE / 32; ++i)
+              load_cw<C>(cbv + (static_cast<size_t>(j) * kE + lane + 32 * i) * C, cv[jw][i]);
+          }
+        }
         // W[e][j] = 2^-S * sum of the columns c = j (mod J): lane = group, rows warp + kNW*k
         constexpr int NR = kE / kNW;                   // rows per warp
         const float inv = ldexpf(1.f, -S);
@@ -782,15 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         }
         __syncthreads();
         // o[j*C + ch] = sum_e W[e][j] C_V[j][e][ch]: warp -> groups, lane -> rows lane + 32 i
-        constexpr int JPW = (J + kNW - 1) / kNW;
-#pragma unroll 1
+#pragma unroll
         for (int jw = 0; jw < JPW; ++jw) {
           const int j = warp + kNW * jw;
           if (j >= J) break;                           // warp-uniform
-          float cv[kE / 32][C];
-#pragma unroll
-          for (int i = 0; i < kE / 32; ++i)
-            load_cw<C>(cbv + (static_cast<size_t>(j) * kE + lane + 32 * i) * C, cv[i]);
           float acc[C];
 #pragma unroll
           for (int ch = 0; ch < C; ++ch) acc[ch] = 0.f;
@@ -798,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           for (int i = 0; i < kE / 32; ++i) {
             const float h = wt[j * EP + lane + 32 * i];
 #pragma unroll
-            for (int ch = 0; ch < C; ++ch) acc[ch] = fmaf(h, cv[i][ch], acc[ch]);
+            for (int ch = 0; ch < C; ++ch) acc[ch] = fmaf(h, cv[jw][i][ch], acc[ch]);
           }
 #pragma unroll
           for (int ch = 0; ch < C; ++ch) {

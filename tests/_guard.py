@@ -36,8 +36,8 @@ class Guarded:
 
 
 def workspace(nbytes, device="cuda"):
-    """A guarded float32 workspace of at least `nbytes` bytes (NaN-filled)
-    whose status word (its first int32) is zero."""
+    """A guarded float32 decode workspace of at least `nbytes` bytes,
+    NaN-filled, whose status word (its first int32) is zero."""
     g = Guarded((max(nbytes // 4, 1),), torch.float32, fill=float("nan"), device=device)
     g.t[:1].view(torch.int32).zero_()
     return g
