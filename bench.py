@@ -274,19 +274,16 @@ class Workload:
                              self.max_seq_len, lse=self.lse[l, t], stream=stream)
 
     def evict_encode(self, stream):
+        """The tokens leaving the recent window, every layer, loop group and
+        K/V, in one launch."""
         import sub_bit_vq_b200 as L
-        s = self.shape
-        for l in range(s.n_layers):
-            for gamma in range(s.G):
-                for kv in range(2):
-                    L.loopvq_encode(self.cfg, l, gamma, kv, self.evict[l, gamma, kv], None, self.cb,
-                                    self.evict_slots, self.pool, stream=stream)
+        L.loopvq_encode_evict(self.cfg, self.evict, self.cb, self.evict_slots, self.pool, stream=stream)
 
     def launches_per_step(self):
         """Kernels per step: two per decode call (the pair kernel, the
-        streaming kernel) and one per eviction encode."""
+        streaming kernel) and one for the eviction encode."""
         s = self.shape
-        return s.n_loops * s.n_layers * 2 + s.n_layers * s.G * 2
+        return s.n_loops * s.n_layers * 2 + 1
 
     def step(self, stream, events=None):
         s = self.shape

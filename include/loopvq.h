@@ -195,6 +195,26 @@ loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_
                             const int64_t* slot_mapping, uint8_t* pool, void* stream);
 
 /*
+ * The window eviction of one decode step in one launch (airadar.tv, section
+ * "Utilisation": the latest RECENT_TOKENS tokens stay in bf16, so each new
+ * token pushes one token out of the recent window into the quantised cache).
+ * Encodes n_tokens tokens, unweighted, exactly as loopvq_encode would for
+ * every (layer, loop group, K/V) of the configuration: for combination
+ * z = (layer*G + loop_group)*2 + kv the g loop slices are read at
+ *     x + z*g*n_tokens*Hkv*d   as dense bf16 [g][n_tokens][Hkv][d],
+ * i.e. x is [L][G][2][g][n_tokens][Hkv][d], and the indices go to the K
+ * (kv = 0) or V plane of (layer, loop group) at slot_mapping[n] (the same
+ * slot for every layer and group: the page tables are shared; a negative
+ * entry skips the token).
+ *  n_tokens   0 .. 64 (one evicted token per sequence of the batch);
+ *             larger batches return LOOPVQ_ERR_UNSUPPORTED.
+ *  x          16-byte aligned; codebooks and pool as for loopvq_encode.
+ */
+loopvq_status loopvq_encode_evict(const loopvq_config* cfg, int n_tokens, const void* x,
+                                  const float* codebooks, const int64_t* slot_mapping,
+                                  uint8_t* pool, void* stream);
+
+/*
  * One weighted k-means (Lloyd) step on the codebooks of (layer,
  * loop_group_idx, K or V) for every kv-head and channel group: the offline
  * codebook fitting that the abstract's quantiser needs (Fisher-weighted

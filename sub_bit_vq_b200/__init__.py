@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     loopvq_decode_attn_noalloc,
     loopvq_decode_workspace_bytes,
     loopvq_encode,
+    loopvq_encode_evict,
     loopvq_kmeans_assign_bytes,
     loopvq_kmeans_step,
     loopvq_status_string,

@@ -75,6 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.loopvq_cache_layout.argtypes = [cfgp, ctypes.POINTER(_Layout)]
     lib.loopvq_encode.restype = I
     lib.loopvq_encode.argtypes = [cfgp, I, I, I, I, P, I64, I64, P, I64, I64, P, P, P, P]
+    lib.loopvq_encode_evict.restype = I
+    lib.loopvq_encode_evict.argtypes = [cfgp, I, P, P, P, P, P]
     lib.loopvq_decode_workspace_bytes.restype = SZ
     lib.loopvq_decode_workspace_bytes.argtypes = [cfgp, I, I]
     lib.loopvq_decode_attn.restype = I
@@ -95,7 +97,7 @@ def _load() -> ctypes.CDLL:
 
 _lib = _load()
 
-EXPORTED = ("loopvq_status_string", "loopvq_cache_layout", "loopvq_encode",
+EXPORTED = ("loopvq_status_string", "loopvq_cache_layout", "loopvq_encode", "loopvq_encode_evict",
             "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
             "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn",
             "loopvq_kmeans_assign_bytes", "loopvq_kmeans_step")
@@ -190,6 +192,18 @@ def loopvq_encode(cfg: LoopVQConfig, layer: int, loop_group_idx: int, kv: int, x
                             x.stride(0), x.stride(1) if n > 1 else 0, _ptr(w), wl, wt,
                             _ptr(codebooks), _ptr(slot_mapping), _ptr(pool), _stream(stream))
     _check("loopvq_encode", st)
+
+
+def loopvq_encode_evict(cfg: LoopVQConfig, x: torch.Tensor, codebooks: torch.Tensor,
+                        slot_mapping: torch.Tensor, pool: torch.Tensor, stream=None) -> None:
+    """x: dense bf16 ``[L][G][2][g][n][Hkv][d]``, the evicted tokens of every
+    (layer, loop group, K/V); slot_mapping: int64 ``[n]``."""
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be dense bfloat16 [L][G][2][g][n][Hkv][d]")
+    n = x.shape[4]
+    st = _lib.loopvq_encode_evict(cfg.c_ref(), n, _ptr(x), _ptr(codebooks), _ptr(slot_mapping),
+                                  _ptr(pool), _stream(stream))
+    _check("loopvq_encode_evict", st)
 
 
 def _xw_strides(x: torch.Tensor, w: torch.Tensor | None) -> tuple[int, int, int, int]:

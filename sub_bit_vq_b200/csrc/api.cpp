@@ -201,6 +201,25 @@ loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_
   return loopvq::launch_encode(a);
 }
 
+loopvq_status loopvq_encode_evict(const loopvq_config* cfg, int n_tokens, const void* x,
+                                  const float* codebooks, const int64_t* slot_mapping,
+                                  uint8_t* pool, void* stream) {
+  Geometry g;
+  loopvq_status st = loopvq::make_geometry(cfg, &g);
+  if (st != LOOPVQ_OK) return st;
+  if (n_tokens < 0) return LOOPVQ_ERR_INVALID_ARG;
+  if (n_tokens == 0) return LOOPVQ_OK;
+  if (n_tokens > 64) return LOOPVQ_ERR_UNSUPPORTED;
+  if (x == nullptr || codebooks == nullptr || slot_mapping == nullptr || pool == nullptr)
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (!loopvq::aligned(x, 16) || !loopvq::aligned(codebooks, 16) || !loopvq::aligned(slot_mapping, 8))
+    return LOOPVQ_ERR_INVALID_ARG;
+  const int64_t n_tok = n_tokens;
+  loopvq::EncodeArgs a{&g, 0, 0, 0, n_tokens, x, n_tok * g.Hkv * g.d, static_cast<int64_t>(g.Hkv) * g.d,
+                       nullptr, 0, 0, codebooks, slot_mapping, pool, nullptr, stream};
+  return loopvq::launch_encode_evict(a);
+}
+
 size_t loopvq_kmeans_assign_bytes(const loopvq_config* cfg, int n_tokens) {
   Geometry g;
   if (loopvq::make_geometry(cfg, &g) != LOOPVQ_OK || n_tokens < 0) return 0;

@@ -30,11 +30,14 @@ constexpr int kEncTcMinTokens = 2048;   // batches from this size take the tenso
 // centroids lane, lane+32, .. with the same float32 weighted distance and
 // term order as encode_kernel, and a shuffle argmin keeps the smallest
 // index among equal distances.
+// The body of the small-batch form for (group j, head h): stages the
+// codebook of (j, h) once as [tau][E][c] in `cbs`; each warp takes tokens
+// warp, warp+8, .., the lanes scan centroids lane, lane+32, .. with the same
+// float32 weighted distance and term order as encode_kernel, and a shuffle
+// argmin keeps the smallest index among equal distances.
 template <int C, int G>
-__global__ void __launch_bounds__(kEncWarpThreads) encode_warp_kernel(const EncodeParams p) {
+__device__ __forceinline__ void encode_tokens_warp(const EncodeParams& p, int j, int h, float* cbs) {
   constexpr int D = C * G;
-  __shared__ __align__(16) float cbs[G * kE * C];
-  const int j = blockIdx.x, h = blockIdx.y;
   const float* cb = p.cb + h * p.cb_stride_head + static_cast<int64_t>(j) * kE * C;
   for (int i = threadIdx.x * 4; i < G * kE * C; i += kEncWarpThreads * 4) {
     const int tau = i / (kE * C), r = i % (kE * C);
@@ -79,6 +82,38 @@ __global__ void __launch_bounds__(kEncWarpThreads) encode_warp_kernel(const Enco
     }
     if (lane == 0) store_index(p, slot, j, h, best_e);
   }
+}
+
+// Small batches (the tokens leaving the recent window at each decode step):
+// one CTA per (group j, head h).
+template <int C, int G>
+__global__ void __launch_bounds__(kEncWarpThreads) encode_warp_kernel(const EncodeParams p) {
+  __shared__ __align__(16) float cbs[G * kE * C];
+  encode_tokens_warp<C, G>(p, blockIdx.x, blockIdx.y, cbs);
+}
+
+// The window eviction of one decode step in one launch: CTA (j, h, z)
+// encodes the tokens for (group j, head h) of combination z = (layer*G +
+// gamma)*2 + kv. Combination z reads its g loop slices at x + z*x_combo
+// ([g][n][Hkv][d] bf16) and writes the K or V plane of (layer, gamma).
+struct EvictParams {
+  EncodeParams base;            // layer 0, gamma 0, K; x of combination 0
+  int64_t x_combo;              // elements between combinations
+  int64_t cb_stride_layer, cb_stride_group, cb_stride_kv;
+  int64_t pool_stride_layer, pool_stride_group;
+  int G;
+};
+
+template <int C, int G>
+__global__ void __launch_bounds__(kEncWarpThreads) encode_evict_kernel(const EvictParams e) {
+  __shared__ __align__(16) float cbs[G * kE * C];
+  const int z = blockIdx.z, kv = z & 1, gamma = (z >> 1) % e.G, layer = (z >> 1) / e.G;
+  EncodeParams p = e.base;
+  p.x = e.base.x + z * e.x_combo;
+  p.cb = e.base.cb + layer * e.cb_stride_layer + gamma * e.cb_stride_group + kv * e.cb_stride_kv;
+  p.pool = e.base.pool + layer * e.pool_stride_layer + gamma * e.pool_stride_group;
+  p.kv = kv;
+  encode_tokens_warp<C, G>(p, blockIdx.x, blockIdx.y, cbs);
 }
 
 template <int C, int G>
@@ -138,7 +173,41 @@ loopvq_status launch_enc(const EncodeParams& p, int J, int H, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
 }
 
+template <int C, int G>
+loopvq_status launch_evict(const EvictParams& e, int J, int H, int combos, cudaStream_t st) {
+  encode_evict_kernel<C, G><<<dim3(J, H, combos), kEncWarpThreads, 0, st>>>(e);
+  return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+}
+
 }  // namespace
+
+loopvq_status launch_encode_evict(const EncodeArgs& a) {
+  const Geometry& g = *a.geo;
+  if (a.n_tokens > kEncWarpMaxTokens) return LOOPVQ_ERR_UNSUPPORTED;
+  EvictParams e{};
+  e.base = encode_params(a);                           // layer 0, gamma 0, K
+  e.x_combo = static_cast<int64_t>(g.g) * a.n_tokens * g.Hkv * g.d;
+  e.cb_stride_layer = g.cb_stride_layer;
+  e.cb_stride_group = g.cb_stride_group;
+  e.cb_stride_kv = g.cb_stride_kv;
+  e.pool_stride_layer = g.pool_stride_layer;
+  e.pool_stride_group = g.pool_stride_group;
+  e.G = g.G;
+  const int combos = g.L * g.G * 2;
+  cudaStream_t st = static_cast<cudaStream_t>(a.stream);
+  switch (g.c * 100 + g.g) {
+    case 404: return launch_evict<4, 4>(e, g.J, g.Hkv, combos, st);
+    case 804: return launch_evict<8, 4>(e, g.J, g.Hkv, combos, st);
+    case 204: return launch_evict<2, 4>(e, g.J, g.Hkv, combos, st);
+    case 402: return launch_evict<4, 2>(e, g.J, g.Hkv, combos, st);
+    case 802: return launch_evict<8, 2>(e, g.J, g.Hkv, combos, st);
+    case 208: return launch_evict<2, 8>(e, g.J, g.Hkv, combos, st);
+    case 408: return launch_evict<4, 8>(e, g.J, g.Hkv, combos, st);
+    case 401: return launch_evict<4, 1>(e, g.J, g.Hkv, combos, st);
+    case 801: return launch_evict<8, 1>(e, g.J, g.Hkv, combos, st);
+    default: return LOOPVQ_ERR_UNSUPPORTED;
+  }
+}
 
 EncodeParams encode_params(const EncodeArgs& a) {
   const Geometry& g = *a.geo;

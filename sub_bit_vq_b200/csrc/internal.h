@@ -78,6 +78,12 @@ struct EncodeArgs {
 };
 loopvq_status launch_encode(const EncodeArgs& a);
 
+// The window eviction of one decode step: every (layer, loop group, K/V)
+// of the config in one launch; x of combination z = (layer*G + gamma)*2 + kv
+// at a.x + z * g*n*Hkv*d elements, dense [g][n][Hkv][d]; unweighted;
+// n_tokens <= 64. a.layer, a.gamma and a.kv are 0.
+loopvq_status launch_encode_evict(const EncodeArgs& a);
+
 // Weighted centroid update of one k-means step: every codebook (h, j) of
 // (layer, gamma, kv) becomes the per-element weighted mean of the
 // sub-vectors assigned to each centroid (assignment [Hkv][J][n_tokens]);

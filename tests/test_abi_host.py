@@ -192,7 +192,8 @@ def test_status_strings():
 
 
 def test_python_api_exports_the_documented_calls():
-    for name in ("LoopVQConfig", "loopvq_cache_layout", "loopvq_encode", "loopvq_kmeans_assign_bytes",
+    for name in ("LoopVQConfig", "loopvq_cache_layout", "loopvq_encode", "loopvq_encode_evict",
+                 "loopvq_kmeans_assign_bytes",
                  "loopvq_kmeans_step", "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
                  "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn",
                  "loopvq_decode_attn_noalloc", "loopvq_status_string"):
@@ -218,3 +219,16 @@ def test_status_bits_match_the_header():
         m = re.search(name + r"\s*=\s*(\d+)", text)
         assert m, name
         assert getattr(B, name) == int(m.group(1)) == getattr(L, name)
+
+
+def test_encode_evict_rejects_before_launch():
+    cfg = _cfg()
+    lib = B.library()
+    E = B.LOOPVQ_ERR_INVALID_ARG
+    ev = lambda n=4, x=0x1000, cb=0x2000, sl=0x3000, pool=0x4000: lib.loopvq_encode_evict(
+        cfg.c_ref(), n, x, cb, sl, pool, None)
+    assert ev(n=0) == B.LOOPVQ_OK                     # nothing to do, nothing launched
+    assert ev(n=-1) == E
+    assert ev(n=65) == B.LOOPVQ_ERR_UNSUPPORTED
+    assert ev(x=0) == E and ev(cb=0) == E and ev(sl=0) == E and ev(pool=0) == E
+    assert ev(x=0x1008) == E and ev(cb=0x2004) == E and ev(sl=0x3004) == E

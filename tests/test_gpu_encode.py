@@ -271,3 +271,39 @@ def test_prefill_tensor_core_d8():
     _, dist = O.encode_group_ref(x.double().numpy(), cb[0, :, 0, 0].double().numpy(),
                                  w.double().numpy())
     check_indices(_gpu_indices(pool, s, 0, 0, 0, slots), dist)
+
+
+def test_eviction_encode_of_every_layer_group_and_plane_in_one_launch():
+    # The one-launch eviction encode writes, for every (layer, loop group,
+    # K/V), exactly the bytes that loopvq_encode writes for that combination
+    # (the same float32 arithmetic), and those indices are the oracle's
+    # nearest centroids; skipped slots and every other byte stay untouched.
+    s = Shape("evict", n_layers=2, n_kv_heads=2, n_q_heads=2, head_dim=64, n_loops=8,
+              loop_group=4, chan_group=4, batch=1, context=0, seed=210)
+    L_, G, n, n_pages = 2, s.G, 12, 4
+    cfg = _cfg(s, L_, n_pages)
+    cb = random_codebooks(s, L_, 211)
+    xs = torch.stack([torch.stack([torch.stack([loop_group_kv(s, l, gm, kv, n, stream=3)
+                                                for kv in range(2)]) for gm in range(G)])
+                      for l in range(L_)])                         # [L][G][2][g][n][H][d]
+    slots = _slots(n, n_pages, s.page_tokens, 212, skip_every=5)
+    pool = Guarded((L_, s.n_kv_heads, G, n_pages, 2, s.page_tokens * s.J), torch.uint8, fill=0)
+    L.loopvq_encode_evict(cfg, xs.cuda(), cb.cuda(), torch.as_tensor(slots).cuda(), pool.t)
+    pool.check("pool")
+    got = pool.t.cpu().numpy()
+    ref = torch.zeros_like(pool.t)
+    for l in range(L_):
+        for gm in range(G):
+            for kv in range(2):
+                L.loopvq_encode(cfg, l, gm, kv, xs[l, gm, kv].cuda(), None, cb.cuda(),
+                                torch.as_tensor(slots).cuda(), ref)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(got, ref.cpu().numpy())
+    keep = slots >= 0
+    for l in range(L_):
+        for gm in range(G):
+            for kv in range(2):
+                _, dist = O.encode_group_ref(xs[l, gm, kv].double().numpy(),
+                                             cb[l, :, gm, kv].double().numpy())
+                idx = _gpu_indices(got, s, l, gm, kv, slots)
+                check_indices(idx[keep], dist[keep])
