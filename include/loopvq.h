@@ -52,6 +52,20 @@ typedef enum {
 
 enum { LOOPVQ_DTYPE_BF16 = 0, LOOPVQ_DTYPE_F32 = 1 };
 
+/* Flag bits of the encoder's status word (per device, see
+ * loopvq_encode_status). */
+enum {
+  /* a tensor-core encode gave up waiting for a tile's tensor-core result:
+   * the tokens of that tile and of the CTA's later tiles were not written */
+  LOOPVQ_ENCODE_STATUS_TIMEOUT = 1,
+  /* ... and its last tensor-core operation did not finish within the
+   * second, longer wait either */
+  LOOPVQ_ENCODE_STATUS_UNDRAINED = 2,
+  /* a slot_mapping entry at or past n_pages * page_tokens: that token was
+   * not written */
+  LOOPVQ_ENCODE_STATUS_BAD_SLOT = 4
+};
+
 /* Flag bits of a decode call's status word (the first int32 of its
  * workspace), set by the kernels, never cleared by them. */
 enum {
@@ -62,7 +76,11 @@ enum {
    * address arithmetic needs it; its records are NaN (the host checks this
    * before launching and returns LOOPVQ_ERR_UNSUPPORTED, so this bit means a
    * device that changed under the library) */
-  LOOPVQ_DECODE_STATUS_SHARED_BASE = 2
+  LOOPVQ_DECODE_STATUS_SHARED_BASE = 2,
+  /* a range check of a build with LOOPVQ_RANGE_CHECK defined found an index
+   * outside its buffer; the access was skipped (never set by the default
+   * build, whose indices are in range by construction) */
+  LOOPVQ_DECODE_STATUS_RANGE = 4
 };
 
 /*
@@ -193,6 +211,16 @@ loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_
                             int64_t x_token_stride, const float* w, int64_t w_loop_stride,
                             int64_t w_token_stride, const float* codebooks,
                             const int64_t* slot_mapping, uint8_t* pool, void* stream);
+
+/*
+ * Reads the encoder status word of the current device into *flags
+ * (LOOPVQ_ENCODE_STATUS_* bits that any loopvq_encode, loopvq_encode_evict or
+ * loopvq_kmeans_step kernel set since the word was last cleared) and clears
+ * it when `clear` is nonzero. This call synchronises with the device (it
+ * copies a device word to the host). A word of zero means every encode so
+ * far wrote all of its indices.
+ */
+loopvq_status loopvq_encode_status(int* flags, int clear);
 
 /*
  * The window eviction of one decode step in one launch (airadar.tv, section

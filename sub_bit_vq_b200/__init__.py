@@ -6,6 +6,10 @@ raises ``ImportError``: there is no CPU fallback.
 """
 from .binding import (  # noqa: F401
     LOOPVQ_DECODE_STATUS_BAD_PAGE,
+    LOOPVQ_ENCODE_STATUS_TIMEOUT,
+    LOOPVQ_ENCODE_STATUS_UNDRAINED,
+    LOOPVQ_ENCODE_STATUS_BAD_SLOT,
+    LOOPVQ_DECODE_STATUS_RANGE,
     LOOPVQ_DECODE_STATUS_SHARED_BASE,
     LOOPVQ_DTYPE_BF16,
     LOOPVQ_DTYPE_F32,
@@ -20,6 +24,7 @@ from .binding import (  # noqa: F401
     loopvq_decode_workspace_bytes,
     loopvq_encode,
     loopvq_encode_evict,
+    loopvq_encode_status,
     loopvq_kmeans_assign_bytes,
     loopvq_kmeans_step,
     loopvq_status_string,

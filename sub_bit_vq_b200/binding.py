@@ -16,7 +16,9 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libloopvq.so")
+# LOOPVQ_LIB names another in-tree build of the same sources (a test build
+# such as libloopvq_rangecheck.so); the default is libloopvq.so.
+LIB_PATH = os.path.join(_HERE, os.environ.get("LOOPVQ_LIB", "libloopvq.so"))
 
 LOOPVQ_OK = 0
 LOOPVQ_ERR_INVALID_ARG = 1
@@ -25,8 +27,12 @@ LOOPVQ_ERR_WORKSPACE = 3
 LOOPVQ_ERR_CUDA = 4
 LOOPVQ_DTYPE_BF16 = 0
 LOOPVQ_DTYPE_F32 = 1
+LOOPVQ_ENCODE_STATUS_TIMEOUT = 1
+LOOPVQ_ENCODE_STATUS_UNDRAINED = 2
+LOOPVQ_ENCODE_STATUS_BAD_SLOT = 4
 LOOPVQ_DECODE_STATUS_BAD_PAGE = 1
 LOOPVQ_DECODE_STATUS_SHARED_BASE = 2
+LOOPVQ_DECODE_STATUS_RANGE = 4
 
 
 class LoopVQError(RuntimeError):
@@ -62,10 +68,10 @@ class _Layout(ctypes.Structure):
     ]
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libloopvq.so not built ({LIB_PATH}); run python sub_bit_vq_b200/build.py")
-    lib = ctypes.CDLL(LIB_PATH)
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not built ({path}); run python sub_bit_vq_b200/build.py")
+    lib = ctypes.CDLL(path)
     P, I, I64, F, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
                         ctypes.c_size_t)
     cfgp = ctypes.POINTER(_Config)
@@ -75,6 +81,8 @@ def _load() -> ctypes.CDLL:
     lib.loopvq_cache_layout.argtypes = [cfgp, ctypes.POINTER(_Layout)]
     lib.loopvq_encode.restype = I
     lib.loopvq_encode.argtypes = [cfgp, I, I, I, I, P, I64, I64, P, I64, I64, P, P, P, P]
+    lib.loopvq_encode_status.restype = I
+    lib.loopvq_encode_status.argtypes = [ctypes.POINTER(ctypes.c_int), I]
     lib.loopvq_encode_evict.restype = I
     lib.loopvq_encode_evict.argtypes = [cfgp, I, P, P, P, P, P]
     lib.loopvq_decode_workspace_bytes.restype = SZ
@@ -98,6 +106,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 EXPORTED = ("loopvq_status_string", "loopvq_cache_layout", "loopvq_encode", "loopvq_encode_evict",
+            "loopvq_encode_status",
             "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
             "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn",
             "loopvq_kmeans_assign_bytes", "loopvq_kmeans_step")
@@ -105,6 +114,12 @@ EXPORTED = ("loopvq_status_string", "loopvq_cache_layout", "loopvq_encode", "loo
 
 def library() -> ctypes.CDLL:
     return _lib
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Another build of the library (e.g. a test build), with the same
+    argument types declared."""
+    return _load(path)
 
 
 @dataclass(frozen=True)
@@ -192,6 +207,14 @@ def loopvq_encode(cfg: LoopVQConfig, layer: int, loop_group_idx: int, kv: int, x
                             x.stride(0), x.stride(1) if n > 1 else 0, _ptr(w), wl, wt,
                             _ptr(codebooks), _ptr(slot_mapping), _ptr(pool), _stream(stream))
     _check("loopvq_encode", st)
+
+
+def loopvq_encode_status(clear: bool = False) -> int:
+    """The encoder status word of the current device (LOOPVQ_ENCODE_STATUS_*
+    bits); synchronises with the device."""
+    v = ctypes.c_int(0)
+    _check("loopvq_encode_status", _lib.loopvq_encode_status(ctypes.byref(v), int(clear)))
+    return v.value
 
 
 def loopvq_encode_evict(cfg: LoopVQConfig, x: torch.Tensor, codebooks: torch.Tensor,

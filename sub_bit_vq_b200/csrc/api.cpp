@@ -201,6 +201,11 @@ loopvq_status loopvq_encode(const loopvq_config* cfg, int layer, int loop_group_
   return loopvq::launch_encode(a);
 }
 
+loopvq_status loopvq_encode_status(int* flags, int clear) {
+  if (flags == nullptr) return LOOPVQ_ERR_INVALID_ARG;
+  return loopvq::encode_status(flags, clear);
+}
+
 loopvq_status loopvq_encode_evict(const loopvq_config* cfg, int n_tokens, const void* x,
                                   const float* codebooks, const int64_t* slot_mapping,
                                   uint8_t* pool, void* stream) {

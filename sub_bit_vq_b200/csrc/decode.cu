@@ -83,6 +83,15 @@ constexpr uint32_t kLutAbs = kSBase + kSmallBytes;        // [E][64] floats, 256
 constexpr uint32_t kHistAbs = kLutAbs + kE * kCols * 4;   // [E][64] 32-bit words, 256-byte rows
 constexpr uint32_t kDynBytes = kHistAbs + kE * kCols * 4 - kSBase;
 
+// A build with LOOPVQ_RANGE_CHECK defined checks, before each access that
+// the partition's arithmetic keeps in range, that it is in range, and
+// flags LOOPVQ_DECODE_STATUS_RANGE (skipping the access) if it is not.
+#ifdef LOOPVQ_RANGE_CHECK
+constexpr bool kRangeCheck = true;
+#else
+constexpr bool kRangeCheck = false;
+#endif
+
 // Bits of the status word (see loopvq.h).
 constexpr int kStatusBadPage = LOOPVQ_DECODE_STATUS_BAD_PAGE;
 constexpr int kStatusSharedBase = LOOPVQ_DECODE_STATUS_SHARED_BASE;
@@ -563,6 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
     const int n_vq = max(0, N - p.W);
     const int pair = b * p.Hq + hq;
     float* rec = p.records + static_cast<size_t>(pair + blockIdx.x) * RS;
+    if (kRangeCheck && (pair + static_cast<int>(blockIdx.x) >= p.B * p.Hq + kMaxStreamCtas ||
+                        static_cast<int>(blockIdx.x) >= kMaxStreamCtas)) {
+      if (tid == 0 && p.status != nullptr) atomicOr(p.status, LOOPVQ_DECODE_STATUS_RANGE);
+      return;                                          // CTA-uniform
+    }
     if (bad_base) {
       if (tid == 0) {
         rec[0] = NAN;
@@ -623,6 +637,10 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           return;
         }
         const int pg = my_first + pi * kNW;
+        if (kRangeCheck && (pg < 0 || pg >= p.max_pages_per_seq || blk >= bpp)) {
+          if (lane == 0 && p.status != nullptr) atomicOr(p.status, LOOPVQ_DECODE_STATUS_RANGE);
+          return;
+        }
         bi.nv = max(0, min(LB, n_vq - pg * p.Pg - blk * LB));
         bi.row = pool_h + static_cast<int64_t>(phys) * p.page_bytes + blk * (LB * J) + lane * T::GR;
       };
@@ -839,6 +857,11 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       const long long u0 = pre * p.Hq + static_cast<long long>(hq) * units_b;
       const int c_first = static_cast<int>(((u0 + 1) * p.n_cta - 1) / U);
       const int c_last = static_cast<int>(((u0 + units_b) * p.n_cta - 1) / U);
+      if (kRangeCheck && (c_first < 0 || c_last >= p.n_cta || c_first > static_cast<int>(blockIdx.x) ||
+                          c_last < static_cast<int>(blockIdx.x))) {
+        if (tid == 0 && p.status != nullptr) atomicOr(p.status, LOOPVQ_DECODE_STATUS_RANGE);
+        return;                                        // CTA-uniform
+      }
       ensure_ready();                                  // the counter was zeroed by the pair kernel
       __threadfence();                                 // this thread's record writes, device-wide
       __syncthreads();

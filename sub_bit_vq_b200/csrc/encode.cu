@@ -230,6 +230,7 @@ EncodeParams encode_params(const EncodeArgs& a) {
   p.page_bytes = g.page_bytes;
   p.plane_bytes = g.plane_bytes;
   p.n_slots = (a.assign != nullptr) ? a.n_tokens : static_cast<int64_t>(g.n_pages) * g.Pg;
+  p.status = encode_status_word();
   p.n_tokens = a.n_tokens;
   p.d = g.d;
   p.Pg = g.Pg;

@@ -21,12 +21,21 @@ struct EncodeParams {
   uint8_t* assign;              // or null: indices [H][J][n_tokens] instead of the pool
   int64_t pool_stride_head, page_bytes, plane_bytes;
   int64_t n_slots;              // n_pages * Pg
+  int* status;                  // the device's encoder status word
   int n_tokens, d, Pg, J, LB, GR, kv;
 };
 
+// Device address of this device's encoder status word (looked up once per
+// device with that device current); null if the runtime fails.
+int* encode_status_word();
+
 // Slot of token n: its pool slot, or n itself when indices go to `assign`.
+// A slot at or past n_slots is not written and flags the encoder status word
+// (a negative one only means "skip this token").
 __device__ __forceinline__ int64_t token_slot(const EncodeParams& p, int n) {
-  return p.slot_mapping != nullptr ? p.slot_mapping[n] : static_cast<int64_t>(n);
+  const int64_t s = p.slot_mapping != nullptr ? p.slot_mapping[n] : static_cast<int64_t>(n);
+  if (s >= p.n_slots && p.status != nullptr) atomicOr(p.status, LOOPVQ_ENCODE_STATUS_BAD_SLOT);
+  return s;
 }
 
 // Writes index `e` of (slot, group j, head h) to its byte in the pool, or to

@@ -30,15 +30,26 @@
 
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "encode_common.cuh"
 
 namespace loopvq {
+
+// Encoder status word of this device (flag bits, LOOPVQ_ENCODE_STATUS_*),
+// set by the kernels and read (and cleared) by loopvq_encode_status.
+__device__ int g_encode_status = 0;
+
 namespace {
 
 constexpr int kTcRows = 128;              // tokens per tile (MMA M)
 constexpr int kTcThreads = 128;           // one thread per tile row
-constexpr int kTcSpin = 1 << 20;          // bounded mbarrier wait
+#ifndef LOOPVQ_TC_SPIN
+#define LOOPVQ_TC_SPIN (1 << 20)
+#endif
+constexpr int kTcSpin = LOOPVQ_TC_SPIN;   // bounded mbarrier wait (tries) for a tile's MMA
+constexpr int kTcDrainSpin = 1 << 24;     // bounded wait for the last MMA before TMEM is freed
 
 template <int C, int G>
 struct TcGeo {
@@ -180,6 +191,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
   const uint32_t my_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const int n_tiles = (p.n_tokens + kTcRows - 1) / kTcRows;
   bool failed = false;
+  int last_phase = 0;                                // parity of the MMA commit a failed wait left behind
   // this thread's token of the next tile, requested one tile ahead
   float s_nx[D], w_nx[D];
   int64_t slot_nx = -1;
@@ -236,7 +248,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
                    ::"r"(mbar_a) : "memory");
     }
     fetch(t + 1);                                    // lands while the tensor cores work
-    bool done = failed;
+    bool done = false;
     for (int it = 0; it < kTcSpin && !done; ++it) {
       uint32_t ok;
       asm volatile(
@@ -245,7 +257,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
           : "=r"(ok) : "r"(mbar_a), "r"(static_cast<uint32_t>(t & 1)) : "memory");
       done = ok != 0u;
     }
-    if (!done) failed = true;                        // no more waits; results below are not stored
+    if (__syncthreads_or(!done)) {                   // CTA-uniform: a thread gave up on this tile
+      failed = true;
+      last_phase = t & 1;
+      break;                                         // nothing of this tile or later is stored
+    }
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
     // ---- this row's minimum, then the exact rescore within the margin ----------
@@ -307,9 +323,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
         }
       }
     }
-    if (live && !failed) store_index(p, slot, j, h, best_e);
+    if (live) store_index(p, slot, j, h, best_e);
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();                                 // TMEM read, A free for the next tile
+  }
+  if (failed) {
+    // the abandoned tile's MMAs still write TMEM: wait (bounded) for their
+    // commit before TMEM is freed, and report the failure
+    if (tid == 0) {
+      bool done = false;
+      for (int it = 0; it < kTcDrainSpin && !done; ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n .reg .pred P;\n mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, P;\n}\n"
+            : "=r"(ok) : "r"(mbar_a), "r"(static_cast<uint32_t>(last_phase)) : "memory");
+        done = ok != 0u;
+      }
+      if (p.status != nullptr)
+        atomicOr(p.status, done ? LOOPVQ_ENCODE_STATUS_TIMEOUT
+                                : (LOOPVQ_ENCODE_STATUS_TIMEOUT | LOOPVQ_ENCODE_STATUS_UNDRAINED));
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
   }
   if (warp == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -332,6 +368,31 @@ loopvq_status launch_tc(const EncodeParams& p, int J, int H, cudaStream_t st) {
 }
 
 }  // namespace
+
+int* encode_status_word() {
+  static std::mutex mu;
+  static int* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_encode_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(a);
+  }
+  return addr[dev];
+}
+
+loopvq_status encode_status(int* flags, int clear) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_encode_status, sizeof(int)) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_encode_status, &zero, sizeof(int)) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+  }
+  *flags = v;
+  return LOOPVQ_OK;
+}
 
 bool encode_tc_supported(int c, int g) {
   const int d = c * g;

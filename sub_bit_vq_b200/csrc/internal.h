@@ -78,6 +78,10 @@ struct EncodeArgs {
 };
 loopvq_status launch_encode(const EncodeArgs& a);
 
+// Reads (and optionally clears) the encoder status word of the current
+// device; synchronous.
+loopvq_status encode_status(int* flags, int clear);
+
 // The window eviction of one decode step: every (layer, loop group, K/V)
 // of the config in one launch; x of combination z = (layer*G + gamma)*2 + kv
 // at a.x + z * g*n*Hkv*d elements, dense [g][n][Hkv][d]; unweighted;

@@ -215,7 +215,9 @@ def test_static_scratch_size_matches_the_header():
 
 def test_status_bits_match_the_header():
     text = open(os.path.join(ROOT, "include", "loopvq.h")).read()
-    for name in ("LOOPVQ_DECODE_STATUS_BAD_PAGE", "LOOPVQ_DECODE_STATUS_SHARED_BASE"):
+    for name in ("LOOPVQ_DECODE_STATUS_BAD_PAGE", "LOOPVQ_DECODE_STATUS_SHARED_BASE",
+                 "LOOPVQ_ENCODE_STATUS_TIMEOUT", "LOOPVQ_ENCODE_STATUS_UNDRAINED",
+                 "LOOPVQ_ENCODE_STATUS_BAD_SLOT", "LOOPVQ_DECODE_STATUS_RANGE"):
         m = re.search(name + r"\s*=\s*(\d+)", text)
         assert m, name
         assert getattr(B, name) == int(m.group(1)) == getattr(L, name)
@@ -232,3 +234,7 @@ def test_encode_evict_rejects_before_launch():
     assert ev(n=65) == B.LOOPVQ_ERR_UNSUPPORTED
     assert ev(x=0) == E and ev(cb=0) == E and ev(sl=0) == E and ev(pool=0) == E
     assert ev(x=0x1008) == E and ev(cb=0x2004) == E and ev(sl=0x3004) == E
+
+
+def test_encode_status_rejects_a_null_pointer():
+    assert B.library().loopvq_encode_status(None, 0) == B.LOOPVQ_ERR_INVALID_ARG

@@ -307,3 +307,25 @@ def test_eviction_encode_of_every_layer_group_and_plane_in_one_launch():
                                              cb[l, :, gm, kv].double().numpy())
                 idx = _gpu_indices(got, s, l, gm, kv, slots)
                 check_indices(idx[keep], dist[keep])
+
+
+def test_slots_past_the_pool_are_skipped_and_flagged():
+    # A slot_mapping entry at or past n_pages * page_tokens is not written and
+    # sets LOOPVQ_ENCODE_STATUS_BAD_SLOT; a negative one is a plain skip.
+    s = SHAPES["tiny"]
+    n, n_pages = 40, 2
+    cfg = _cfg(s, 1, n_pages)
+    cb = random_codebooks(s, 1, 213)
+    x = loop_group_kv(s, 0, 0, 0, n, stream=5)
+    slots = _slots(n, n_pages, s.page_tokens, 214)
+    slots[3] = n_pages * s.page_tokens          # one past the pool
+    slots[7] = -1
+    L.loopvq_encode_status(clear=True)
+    pool = _run(s, 1, 0, 0, 0, x, None, cb, slots, n_pages)
+    assert L.loopvq_encode_status(clear=True) & L.LOOPVQ_ENCODE_STATUS_BAD_SLOT
+    ok = np.ones(n, dtype=bool)
+    ok[[3, 7]] = False
+    _, dist = O.encode_group_ref(x.double().numpy(), cb[0, :, 0, 0].double().numpy())
+    idx = _gpu_indices(pool, s, 0, 0, 0, np.where(ok, slots, -1))
+    check_indices(idx[ok], dist[ok])
+    assert L.loopvq_encode_status() == 0        # cleared
