@@ -325,6 +325,36 @@ loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_s
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Attention of a chunk of new queries over the cached context (the prefill
+ * or chunked-prefill side of the same cache; airadar.tv, section
+ * "Utilisation", names the prefill backend as a serving setting). For each
+ * sequence b and each of its n_queries queries i, computes exactly what
+ * loopvq_decode_attn computes for a single query: attention of
+ * q[b][i][hq] over the min(N, P+R) window tokens and the N-P-R quantised
+ * tokens of sequence b, N = seq_lens[b]. Attention among the chunk's own
+ * tokens (causal, not yet cached) is the caller's; out and lse are returned
+ * so that the caller merges the two with log-sum-exp weights.
+ *
+ *  q      bf16 [batch][n_queries][Hq][d], 16-byte aligned.
+ *  out    [batch][n_queries][Hq][d] (bf16 or float32 as out_dtype).
+ *  lse    float32 [batch][n_queries][Hq] or NULL.
+ *  workspace  at least loopvq_prefill_workspace_bytes(cfg, batch, n_queries,
+ *         max_seq_len) bytes; the status word as for loopvq_decode_attn.
+ * Every other argument as for loopvq_decode_attn. The queries of a
+ * sequence are streamed by neighbouring CTAs, so each index page crosses
+ * HBM about once and is reused from L2.
+ */
+size_t loopvq_prefill_workspace_bytes(const loopvq_config* cfg, int batch, int n_queries,
+                                      int max_seq_len);
+loopvq_status loopvq_prefill_attn(const loopvq_config* cfg, int layer, int loop_step, int batch,
+                                  int n_queries, int max_seq_len, const void* q,
+                                  const uint8_t* pool, const float* codebooks,
+                                  const int32_t* block_table, const int32_t* seq_lens,
+                                  const void* win_k, const void* win_v, float sm_scale,
+                                  int out_dtype, void* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
  * Decode attention that needs no workspace from the caller. The pages have
  * no counterpart for this call; it exists for callers that cannot allocate
  * device memory: code that receives only input and output pointers from a

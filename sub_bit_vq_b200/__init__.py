@@ -27,5 +27,7 @@ from .binding import (  # noqa: F401
     loopvq_encode_status,
     loopvq_kmeans_assign_bytes,
     loopvq_kmeans_step,
+    loopvq_prefill_attn,
+    loopvq_prefill_workspace_bytes,
     loopvq_status_string,
 )

@@ -85,6 +85,11 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.loopvq_encode_status.argtypes = [ctypes.POINTER(ctypes.c_int), I]
     lib.loopvq_encode_evict.restype = I
     lib.loopvq_encode_evict.argtypes = [cfgp, I, P, P, P, P, P]
+    lib.loopvq_prefill_workspace_bytes.restype = SZ
+    lib.loopvq_prefill_workspace_bytes.argtypes = [cfgp, I, I, I]
+    lib.loopvq_prefill_attn.restype = I
+    lib.loopvq_prefill_attn.argtypes = [cfgp, I, I, I, I, I, P, P, P, P, P, P, P, F, I, P, P, P, SZ,
+                                        P]
     lib.loopvq_decode_workspace_bytes.restype = SZ
     lib.loopvq_decode_workspace_bytes.argtypes = [cfgp, I, I]
     lib.loopvq_decode_attn.restype = I
@@ -106,7 +111,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
 _lib = _load()
 
 EXPORTED = ("loopvq_status_string", "loopvq_cache_layout", "loopvq_encode", "loopvq_encode_evict",
-            "loopvq_encode_status",
+            "loopvq_encode_status", "loopvq_prefill_workspace_bytes", "loopvq_prefill_attn",
             "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
             "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn",
             "loopvq_kmeans_assign_bytes", "loopvq_kmeans_step")
@@ -287,6 +292,31 @@ def loopvq_decode_attn(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.T
         float(sm_scale), odt, _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("loopvq_decode_attn", st)
+
+
+def loopvq_prefill_workspace_bytes(cfg: LoopVQConfig, batch: int, n_queries: int,
+                                   max_seq_len: int) -> int:
+    return int(_lib.loopvq_prefill_workspace_bytes(cfg.c_ref(), batch, n_queries, max_seq_len))
+
+
+def loopvq_prefill_attn(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.Tensor,
+                        pool: torch.Tensor, codebooks: torch.Tensor, block_table: torch.Tensor,
+                        seq_lens: torch.Tensor, win_k: torch.Tensor, win_v: torch.Tensor,
+                        out: torch.Tensor, workspace: torch.Tensor, max_seq_len: int,
+                        lse: torch.Tensor | None = None, sm_scale: float | None = None,
+                        stream=None) -> None:
+    """q: bf16 ``[B][Q][Hq][d]``; out ``[B][Q][Hq][d]``; lse ``[B][Q][Hq]``."""
+    batch, nq = q.shape[0], q.shape[1]
+    if sm_scale is None:
+        sm_scale = cfg.head_dim ** -0.5
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    odt = LOOPVQ_DTYPE_F32 if out.dtype == torch.float32 else LOOPVQ_DTYPE_BF16
+    st = _lib.loopvq_prefill_attn(
+        cfg.c_ref(), layer, loop_step, batch, nq, max_seq_len, _ptr(q), _ptr(pool), _ptr(codebooks),
+        _ptr(block_table), _ptr(seq_lens), _ptr(win_k), _ptr(win_v), float(sm_scale), odt, _ptr(out),
+        _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("loopvq_prefill_attn", st)
 
 
 LOOPVQ_STATIC_SCRATCH_BYTES = 16 << 20

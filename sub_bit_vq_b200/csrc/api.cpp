@@ -259,45 +259,87 @@ loopvq_status loopvq_kmeans_step(const loopvq_config* cfg, int layer, int loop_g
   return loopvq::launch_kmeans_update(a, codebooks);   // weighted means, in place
 }
 
-loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_step, int batch,
-                                 int max_seq_len, const void* q, const uint8_t* pool,
-                                 const float* codebooks, const int32_t* block_table,
-                                 const int32_t* seq_lens, const void* win_k, const void* win_v,
-                                 float sm_scale, int out_dtype, void* out, float* lse,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace loopvq {
+namespace {
+
+// Checks and launches a decode of n_queries queries per sequence (decode:
+// 1; prefill over the cache: a chunk of queries).
+loopvq_status decode_common(const loopvq_config* cfg, int layer, int loop_step, int batch,
+                            int n_queries, int max_seq_len, const void* q, const uint8_t* pool,
+                            const float* codebooks, const int32_t* block_table,
+                            const int32_t* seq_lens, const void* win_k, const void* win_v,
+                            float sm_scale, int out_dtype, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
   Geometry g;
-  loopvq_status st = loopvq::make_geometry(cfg, &g);
+  loopvq_status st = make_geometry(cfg, &g);
   if (st != LOOPVQ_OK) return st;
   if (layer < 0 || layer >= g.L || loop_step < 0 || loop_step >= g.T) return LOOPVQ_ERR_INVALID_ARG;
-  if (batch <= 0 || batch > g.max_batch || max_seq_len < 0) return LOOPVQ_ERR_INVALID_ARG;
+  if (batch <= 0 || batch > g.max_batch || max_seq_len < 0 || n_queries <= 0) return LOOPVQ_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * n_queries * g.Hq > (1ll << 30)) return LOOPVQ_ERR_UNSUPPORTED;
   if (out_dtype != LOOPVQ_DTYPE_BF16 && out_dtype != LOOPVQ_DTYPE_F32) return LOOPVQ_ERR_INVALID_ARG;
   if (!(sm_scale > 0.0f) || sm_scale > 1e30f) return LOOPVQ_ERR_INVALID_ARG;
   if (q == nullptr || pool == nullptr || codebooks == nullptr || block_table == nullptr ||
       seq_lens == nullptr || out == nullptr || workspace == nullptr)
     return LOOPVQ_ERR_INVALID_ARG;
   if (g.W > 0 && (win_k == nullptr || win_v == nullptr)) return LOOPVQ_ERR_INVALID_ARG;
-  if (!loopvq::aligned(q, 16) || !loopvq::aligned(pool, 16) || !loopvq::aligned(codebooks, 16) ||
-      !loopvq::aligned(block_table, 4) || !loopvq::aligned(seq_lens, 4) ||
-      !loopvq::aligned(workspace, 16) || !loopvq::aligned(out, 16) ||
-      (lse != nullptr && !loopvq::aligned(lse, 4)))
+  if (!aligned(q, 16) || !aligned(pool, 16) || !aligned(codebooks, 16) ||
+      !aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(workspace, 16) ||
+      !aligned(out, 16) || (lse != nullptr && !aligned(lse, 4)))
     return LOOPVQ_ERR_INVALID_ARG;
-  if (g.W > 0 && (!loopvq::aligned(win_k, 16) || !loopvq::aligned(win_v, 16)))
-    return LOOPVQ_ERR_INVALID_ARG;
-  const int pages = loopvq::pages_for(g, max_seq_len);
+  if (g.W > 0 && (!aligned(win_k, 16) || !aligned(win_v, 16))) return LOOPVQ_ERR_INVALID_ARG;
+  const int pages = pages_for(g, max_seq_len);
   if (pages > g.max_pages_per_seq) return LOOPVQ_ERR_INVALID_ARG;
-  const size_t need = loopvq_decode_workspace_bytes(cfg, batch, max_seq_len);
+  const size_t need = decode_workspace_bytes(batch * n_queries * g.Hq, g.J, g.d);
   if (workspace_bytes < need) return LOOPVQ_ERR_WORKSPACE;
   loopvq_status err = LOOPVQ_OK;
-  const int sms = loopvq::current_sm_count(&err);
+  const int sms = current_sm_count(&err);
   if (err != LOOPVQ_OK) return err;
   // persistent streaming grid: one CTA per SM, never more CTAs than pages
-  const long long units_max = static_cast<long long>(batch) * g.Hq * pages;
-  int n_cta = sms < loopvq::kMaxStreamCtas ? sms : loopvq::kMaxStreamCtas;
+  const long long units_max = static_cast<long long>(batch) * n_queries * g.Hq * pages;
+  int n_cta = sms < kMaxStreamCtas ? sms : kMaxStreamCtas;
   if (units_max < n_cta) n_cta = static_cast<int>(units_max);
-  loopvq::DecodeArgs a{&g,      layer,  loop_step,  batch,    max_seq_len, q,    pool,
-                       codebooks, block_table, seq_lens, win_k, win_v,      sm_scale, out_dtype,
-                       out,     lse,    workspace,  n_cta,    stream};
-  return loopvq::launch_decode(a);
+  DecodeArgs a{&g,        layer,       loop_step, batch, n_queries, max_seq_len, q,        pool,
+               codebooks, block_table, seq_lens,  win_k, win_v,     sm_scale,    out_dtype, out,
+               lse,       workspace,   n_cta,     stream};
+  return launch_decode(a);
+}
+
+}  // namespace
+}  // namespace loopvq
+
+extern "C" {
+
+loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_step, int batch,
+                                 int max_seq_len, const void* q, const uint8_t* pool,
+                                 const float* codebooks, const int32_t* block_table,
+                                 const int32_t* seq_lens, const void* win_k, const void* win_v,
+                                 float sm_scale, int out_dtype, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return loopvq::decode_common(cfg, layer, loop_step, batch, 1, max_seq_len, q, pool, codebooks,
+                               block_table, seq_lens, win_k, win_v, sm_scale, out_dtype, out, lse,
+                               workspace, workspace_bytes, stream);
+}
+
+size_t loopvq_prefill_workspace_bytes(const loopvq_config* cfg, int batch, int n_queries,
+                                      int max_seq_len) {
+  Geometry g;
+  if (loopvq::make_geometry(cfg, &g) != LOOPVQ_OK || batch <= 0 || n_queries <= 0 || max_seq_len < 0)
+    return 0;
+  return loopvq::decode_workspace_bytes(batch * n_queries * g.Hq, g.J, g.d);
+}
+
+loopvq_status loopvq_prefill_attn(const loopvq_config* cfg, int layer, int loop_step, int batch,
+                                  int n_queries, int max_seq_len, const void* q,
+                                  const uint8_t* pool, const float* codebooks,
+                                  const int32_t* block_table, const int32_t* seq_lens,
+                                  const void* win_k, const void* win_v, float sm_scale,
+                                  int out_dtype, void* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return loopvq::decode_common(cfg, layer, loop_step, batch, n_queries, max_seq_len, q, pool,
+                               codebooks, block_table, seq_lens, win_k, win_v, sm_scale, out_dtype,
+                               out, lse, workspace, workspace_bytes, stream);
 }
 
 size_t loopvq_bf16_decode_workspace_bytes(int batch, int n_q_heads, int head_dim,

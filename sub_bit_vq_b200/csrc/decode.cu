@@ -114,7 +114,10 @@ struct DecodeParams {
   int* status;                      // status word (bit flags), never cleared by the kernels
   void* out;
   float* lse;
-  int B, Hq, Hkv, ratio, W, Pg, n_pages, max_pages_per_seq, max_seq_len;
+  // B counts virtual sequences: sequence b / Q with its query b % Q (Q = 1
+  // for decode); inputs of a sequence (seq_lens, block_table, windows) are
+  // indexed by b / Q, those of a query (q, out, lse) by b.
+  int B, Q, Hq, Hkv, ratio, W, Pg, n_pages, max_pages_per_seq, max_seq_len;
   int64_t page_bytes, plane_bytes;
   int n_cta, out_dtype, log2_bpp;
   float scale_log2;
@@ -222,7 +225,7 @@ __device__ __forceinline__ void red_at(uint32_t a, uint32_t w) {
 
 // Quantised-token pages of sequence b.
 __device__ __forceinline__ int seq_pages(const DecodeParams& p, int b) {
-  const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
+  const int N = max(0, min(p.seq_lens[b / p.Q], p.max_seq_len));
   const int n_vq = max(0, N - p.W);
   return min((n_vq + p.Pg - 1) / p.Pg, p.max_pages_per_seq);
 }
@@ -295,7 +298,7 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
     qf[k][0] = f.x * p.scale_log2;
     qf[k][1] = f.y * p.scale_log2;
   }
-  const size_t head = (static_cast<size_t>(b) * p.Hkv + hkv) * static_cast<size_t>(p.W) * D;
+  const size_t head = (static_cast<size_t>(b / p.Q) * p.Hkv + hkv) * static_cast<size_t>(p.W) * D;
   const unsigned int* wk = reinterpret_cast<const unsigned int*>(p.win_k + head);
   const unsigned int* wv = reinterpret_cast<const unsigned int*>(p.win_v + head);
   float m = -INFINITY, l = 0.f;
@@ -477,7 +480,7 @@ __global__ void __launch_bounds__(kPairThreads) vq_pair_kernel(const DecodeParam
   asm volatile("griddepcontrol.launch_dependents;");
   const int tid = threadIdx.x;
   if (part == 0) {
-    const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
+    const int N = max(0, min(p.seq_lens[b / p.Q], p.max_seq_len));
     window_partial<D, NW>(p, b, hkv, p.q + static_cast<size_t>(pair) * D, min(N, p.W), wst, wpart, wres);
     float* wr = p.wrecs + static_cast<size_t>(pair) * RS;
     for (int i = tid; i < D + 2; i += kPairThreads) wr[i < 2 ? i : i + 2] = wres[i];
@@ -568,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
     const int pg_lo = max(pu_start - kSegmentUnits, 0);
     const int pg_hi = max(pu_start + seg_units - kSegmentUnits, 0);
     const int hkv = hq / p.ratio;
-    const int N = max(0, min(p.seq_lens[b], p.max_seq_len));
+    const int N = max(0, min(p.seq_lens[b / p.Q], p.max_seq_len));
     const int n_vq = max(0, N - p.W);
     const int pair = b * p.Hq + hq;
     float* rec = p.records + static_cast<size_t>(pair + blockIdx.x) * RS;
@@ -602,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       // Chunk ch holds blocks [ch*KB, (ch+1)*KB) of every warp: their key rows,
       // then their value rows.
       const uint8_t* pool_h = p.pool_lg + hkv * p.pool_stride_head;
-      const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages_per_seq;
+      const int32_t* bt = p.block_table + static_cast<size_t>(b / p.Q) * p.max_pages_per_seq;
       auto pages_of = [&](int w) { return (pg_hi > pg_lo + w) ? (pg_hi - pg_lo - w + kNW - 1) / kNW : 0; };
       const int my_first = pg_lo + warp;
       const int n_my_pages = pages_of(warp);
@@ -985,7 +988,7 @@ loopvq_status launch_decode(const DecodeArgs& a) {
   p.win_v = static_cast<const uint16_t*>(a.win_v);
   // workspace: status word, segment records, key lookup tables
   char* ws = static_cast<char*>(a.workspace);
-  const size_t pairs = static_cast<size_t>(a.batch) * g.Hq;
+  const size_t pairs = static_cast<size_t>(a.batch) * a.n_queries * g.Hq;
   p.status = reinterpret_cast<int*>(ws);
   const size_t rec = (4 + static_cast<size_t>(g.d)) * sizeof(float);
   p.records = reinterpret_cast<float*>(ws + kStatusBytes);
@@ -994,7 +997,8 @@ loopvq_status launch_decode(const DecodeArgs& a) {
   p.counts = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(p.luts) + pairs * kE * g.J * sizeof(float));
   p.out = a.out;
   p.lse = a.lse;
-  p.B = a.batch;
+  p.B = a.batch * a.n_queries;
+  p.Q = a.n_queries;
   p.Hq = g.Hq;
   p.Hkv = g.Hkv;
   p.ratio = g.Hq / g.Hkv;

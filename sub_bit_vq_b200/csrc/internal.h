@@ -45,7 +45,7 @@ int current_sm_count(loopvq_status* err);
 // Launchers (defined in the .cu files). All arguments are validated.
 struct DecodeArgs {
   const Geometry* geo;
-  int layer, loop_step, batch, max_seq_len;
+  int layer, loop_step, batch, n_queries, max_seq_len;
   const void* q;
   const uint8_t* pool;
   const float* codebooks;

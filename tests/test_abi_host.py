@@ -238,3 +238,21 @@ def test_encode_evict_rejects_before_launch():
 
 def test_encode_status_rejects_a_null_pointer():
     assert B.library().loopvq_encode_status(None, 0) == B.LOOPVQ_ERR_INVALID_ARG
+
+
+def test_prefill_rejects_before_launch_and_sizes_its_workspace():
+    cfg = _cfg()
+    lib = B.library()
+    need = L.loopvq_prefill_workspace_bytes(cfg, 2, 5, 72 + 5 * 64)
+    assert need == L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64) + \
+        (need - L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64))
+    assert need > L.loopvq_decode_workspace_bytes(cfg, 2, 72 + 5 * 64)
+    assert L.loopvq_prefill_workspace_bytes(cfg, 2, 0, 100) == 0
+
+    def call(nq=5, ws=0x5000, nbytes=need):
+        return lib.loopvq_prefill_attn(cfg.c_ref(), 0, 0, 2, nq, 72 + 5 * 64, 0x1000, 0x2000, 0x3000,
+                                       0x4000, 0x4100, 0x6000, 0x7000, 0.1, 0, 0x8000, None, ws,
+                                       nbytes, None)
+    assert call(nq=0) == B.LOOPVQ_ERR_INVALID_ARG
+    assert call(ws=0) == B.LOOPVQ_ERR_INVALID_ARG
+    assert call(nbytes=need - 1) == B.LOOPVQ_ERR_WORKSPACE
