@@ -556,7 +556,46 @@ def decode_rows(device, peak):
     dp = SHAPES["deep025"]
     rows["deep025"] = decode_row(dp.with_(n_layers=1), [dp.context] * dp.batch, 1,
                                  [0, dp.n_loops - 1], device, peak, l2)
+    rows["prefill"] = prefill_row(device, peak)
     return rows
+
+
+def prefill_row(device, peak, Q=128, B=2):
+    """A chunk of Q = 128 new queries per sequence over a 16384-token cached
+    context (16 heads, d = 128, 0.5 bit), against Q single-query decode
+    calls on the same cache."""
+    import torch
+
+    import sub_bit_vq_b200 as L
+    from synthetic import SHAPES, queries, window_kv
+
+    s = SHAPES["sweep"].with_(batch=B)
+    cfg, pool, cb, bt = encoded_layers(s, 1, [s.context] * B, [0], device)
+    sl = torch.full((B,), s.context, dtype=torch.int32, device=device)
+    g = torch.Generator(device=device).manual_seed(5)
+    q = torch.randn(B, Q, s.n_q_heads, s.head_dim, generator=g, device=device).to(torch.bfloat16)
+    wk, wv = window_kv(s, 0, 0, 0, batch=B, device=device), window_kv(s, 0, 0, 1, batch=B, device=device)
+    out = torch.empty(B, Q, s.n_q_heads, s.head_dim, dtype=torch.bfloat16, device=device)
+    lse = torch.empty(B, Q, s.n_q_heads, device=device)
+    ws = torch.zeros(L.loopvq_prefill_workspace_bytes(cfg, B, Q, s.context) // 4 + 4, device=device)
+    call = lambda st: L.loopvq_prefill_attn(cfg, 0, 0, q, pool, cb, bt, sl, wk, wv, out, ws, s.context,
+                                            lse=lse, stream=st)
+    per, _ = time_calls([call], reps=10)
+    us = statistics.median(per)
+    alg = alg_bytes_per_call(s, [s.context] * B)     # the cache once, plus Q-fold q/out
+    alg += B * (Q - 1) * s.n_q_heads * (s.head_dim * 2 * 2 + 4)
+    # the same queries one decode call at a time
+    qd = q[:, 0].contiguous()
+    outd = torch.empty(B, s.n_q_heads, s.head_dim, dtype=torch.bfloat16, device=device)
+    wsd = torch.zeros(L.loopvq_decode_workspace_bytes(cfg, B, s.context) // 4 + 4, device=device)
+    dcall = lambda st: L.loopvq_decode_attn(cfg, 0, 0, qd, pool, cb, bt, sl, wk, wv, outd, wsd, s.context,
+                                            stream=st)
+    perd, _ = time_calls([dcall], reps=20)
+    return {"batch": B, "queries_per_seq": Q, "context": s.context, "us_per_call": us,
+            "queries_per_s": B * Q * s.n_q_heads / (us * 1e-6), "alg_bytes_per_call": alg,
+            "gbps": alg / us / 1e3, "frac_of_measured_hbm": alg / us / 1e3 / peak,
+            "decode_us_per_query_chunk_of_1": statistics.median(perd),
+            "speedup_vs_q_decode_calls": Q * statistics.median(perd) / us}
 
 
 def encode_prefill(device, reps=3):
