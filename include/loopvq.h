@@ -383,7 +383,7 @@ loopvq_status loopvq_prefill_attn(const loopvq_config* cfg, int layer, int loop_
  * kernels overlap on the GPU, e.g. on two streams without ordering, race
  * on it and give undefined results.
  */
-#define LOOPVQ_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+#define LOOPVQ_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 loopvq_status loopvq_decode_attn_noalloc(const loopvq_config* cfg, int layer, int loop_step,
                                          int batch, int max_seq_len, const void* q,
                                          const uint8_t* pool, const float* codebooks,

@@ -319,7 +319,7 @@ def loopvq_prefill_attn(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.
     _check("loopvq_prefill_attn", st)
 
 
-LOOPVQ_STATIC_SCRATCH_BYTES = 16 << 20
+LOOPVQ_STATIC_SCRATCH_BYTES = 32 << 20
 
 
 def loopvq_decode_attn_noalloc(cfg: LoopVQConfig, layer: int, loop_step: int, q: torch.Tensor,

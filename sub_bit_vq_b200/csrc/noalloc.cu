@@ -15,7 +15,7 @@
 namespace loopvq {
 namespace {
 
-constexpr size_t kStaticScratchBytes = LOOPVQ_STATIC_SCRATCH_BYTES;   // 16 MiB per device
+constexpr size_t kStaticScratchBytes = LOOPVQ_STATIC_SCRATCH_BYTES;   // 32 MiB per device
 
 __device__ __align__(256) float g_decode_scratch[kStaticScratchBytes / sizeof(float)];
 
