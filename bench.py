@@ -629,7 +629,7 @@ def encode_prefill(device, reps=3):
     return {"subvectors_per_s": nsub / sec, "ms_per_call": sec * 1e3,
             "shape": f"{n} tokens x {s.n_kv_heads} heads x {s.J} groups, D={s.D}, "
                      f"per-token LogNormal weights, one of K/V",
-            "kernel": "tcgen05 split-bf16 contraction + exact float32 rescore (tensor cores)",
+            "kernel": "tcgen05 scaled-fp16 contraction + exact float32 rescore (tensor cores)",
             "bounds": encode_bounds(nsub, s.D, sec)}
 
 
@@ -638,8 +638,9 @@ def encode_bounds(nsub: int, D: int, sec: float) -> dict:
     elements with per-token weights, as fractions achieved in `sec`:
     - hbm: bf16 x and float32 w read, one index byte written;
     - tensor: the cross and weight terms of the distance, 2 * (2 D) * 256
-      flops per sub-vector (the algorithmic count; the split-bf16 operands
-      triple the issued work), against the measured bf16 GEMM rate;
+      flops per sub-vector (the algorithmic count, issued as one fp16
+      product per term), against the measured bf16 GEMM rate (fp16 runs
+      at the same rate);
     - alu: 256 candidates x 3 operations (bias add, compare, select) per
       sub-vector, against 148 SMs x 128 float32 lanes x the maximum SM clock."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")

@@ -12,23 +12,32 @@
 // centroids in shared memory and walks the tokens in tiles of 128. For each
 // tile every thread writes its token's row of A, one thread issues the
 // tcgen05.mma chain that leaves S (128 x 256, fp32) in tensor memory, and
-// each thread reads its row back with tcgen05.ld. Operands are bf16 split
-// into high and low parts, a.b ~= a_hi.b_hi + a_hi.b_lo + a_lo.b_hi (K' =
-// 6D): each S_e is off by at most about 2^-14.3 * sum_i |a_i b_ei| (the
-// dropped lo*lo terms, the split residuals, fp32 accumulation over K'), so
-// twice that, plus the direct form's own rounding, stays below
-//     margin = 2^-12 * (sum_i |a_i| max_e |b_ei| + sum_i w_i s_i^2).
-// Every centroid whose S_e is within the margin of the row's minimum is
-// rescored with the float32 direct form and term order of encode_kernel;
-// the first minimum of those (smallest index on equal distances) is the
-// index encode_kernel chooses.
+// each thread reads its row back with tcgen05.ld.
+//
+// Operands are fp16, scaled by powers of two so that each operand uses the
+// top of fp16's range: the -2C half of B by 2^beta1 and the C*C half by
+// 2^beta2 (fixed per codebook), a row of A by 2^(rho - beta) per half (rho
+// per row). Every product of a row is then a_k b_ek 2^rho, so S' = 2^rho S
+// has S's argmin. fp16 x fp16 products are exact in the fp32 accumulator,
+// so with alpha = scaled a and beta' = scaled b, each S'_e is off by at most
+//     2^-9.98 sum_k |alpha_k| |beta'_ek| + 2^-24.9 (sum_k |alpha_k| + sum_k |beta'_ek|)
+// (the two fp16 roundings, 2^-11 each, the float32 rounding of w*s and C*C,
+// fp16's subnormal spacing and the fp32 accumulation over K). Every centroid
+// within
+//     margin = 2^-8.5 2^rho sum_k |a_k| max_e |b_ek| + 2^-17 2^rho sum_i w_i s_i^2
+//              + 2^-23 (sum_k |alpha_k| + sum_k max_e |beta'_ek|)
+// of the row's smallest S'_e is rescored with the float32 direct form and
+// term order of encode_kernel (the margin covers twice the error above plus
+// the direct form's own rounding); the first minimum of those (smallest
+// index on equal distances) is the index encode_kernel chooses. A row whose
+// minimum or margin is not finite rescores all 256 centroids.
 //
 // Shared operands use the K-major layout without swizzle: 8-row x 16-byte
 // core matrices, the two 8-element halves of a 16-wide K step 128 bytes
 // apart (leading byte offset) and consecutive 8-row groups KP*16 bytes
 // apart (stride byte offset).
 
-#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -50,20 +59,25 @@ constexpr int kTcThreads = 128;           // one thread per tile row
 #endif
 constexpr int kTcSpin = LOOPVQ_TC_SPIN;   // bounded mbarrier wait (tries) for a tile's MMA
 constexpr int kTcDrainSpin = 1 << 24;     // bounded wait for the last MMA before TMEM is freed
+constexpr int kTopExp = 13;               // scaled operands lie in [2^13, 2^14) at their largest
+constexpr float kMarginRel = 0.0027621358640099515f;    // 2^-8.5
+constexpr float kMarginWss = 7.62939453125e-06f;        // 2^-17
+constexpr float kMarginAbs = 1.1920928955078125e-07f;   // 2^-23
 
 template <int C, int G>
 struct TcGeo {
   static constexpr int D = C * G;
   static constexpr int K2 = 2 * D;                      // [w*s, w] . [-2C, C*C]
-  static constexpr int KP = ((3 * K2 + 15) / 16) * 16;  // split operands, padded to the MMA K step
+  static constexpr int KP = ((K2 + 15) / 16) * 16;      // padded to the MMA K step
   static constexpr int A_BYTES = kTcRows * KP * 2;
   static constexpr int B_BYTES = kE * KP * 2;
   static constexpr int CB_FLOATS = G * kE * C;          // fp32 codebook [tau][E][c] for rescoring
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = A_OFF + A_BYTES;
   static constexpr int CB_OFF = B_OFF + B_BYTES;
-  static constexpr int BMAX_OFF = CB_OFF + CB_FLOATS * 4;   // [K2] uint (float bits)
-  static constexpr int MBAR_OFF = (BMAX_OFF + K2 * 4 + 7) & ~7;
+  static constexpr int BMAX_OFF = CB_OFF + CB_FLOATS * 4;   // [K2] uint: max_e |b_ek| (float bits)
+  static constexpr int MASK_OFF = BMAX_OFF + K2 * 4;        // [E/32][kTcRows] candidate masks
+  static constexpr int MBAR_OFF = (MASK_OFF + (kE / 32) * kTcRows * 4 + 7) & ~7;
   static constexpr int TMEM_OFF = MBAR_OFF + 8;
   static constexpr int SMEM = TMEM_OFF + 16;
 };
@@ -81,54 +95,130 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, int kp) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3fffu) | (lbo << 16) | (sbo << 32) | (1ull << 46);
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major,
+// Instruction descriptor: f16 x f16 -> fp32, both operands K-major,
 // M = 128, N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdesc = (1u << 4) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
 
 __device__ __forceinline__ uint32_t u32_smem(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-  hi = __float2bfloat16_rn(x);
-  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+// floor(log2 m) for a normal m > 0 (-127 for zero or subnormal m).
+__device__ __forceinline__ int exp_of(float m) {
+  return static_cast<int>((__float_as_uint(m) >> 23) & 0xffu) - 127;
 }
 
-// Writes 8 bf16 values (one 16-byte core-matrix row) at byte offset `off`.
-__device__ __forceinline__ void st_row8(unsigned char* base, uint32_t off, const __nv_bfloat16 (&v)[8]) {
-  uint4 u;
-  u.x = static_cast<uint32_t>(__bfloat16_as_ushort(v[0])) | (static_cast<uint32_t>(__bfloat16_as_ushort(v[1])) << 16);
-  u.y = static_cast<uint32_t>(__bfloat16_as_ushort(v[2])) | (static_cast<uint32_t>(__bfloat16_as_ushort(v[3])) << 16);
-  u.z = static_cast<uint32_t>(__bfloat16_as_ushort(v[4])) | (static_cast<uint32_t>(__bfloat16_as_ushort(v[5])) << 16);
-  u.w = static_cast<uint32_t>(__bfloat16_as_ushort(v[6])) | (static_cast<uint32_t>(__bfloat16_as_ushort(v[7])) << 16);
-  *reinterpret_cast<uint4*>(base + off) = u;
+// 2^e for e in [-126, 127] (clamped), exactly.
+__device__ __forceinline__ float pow2(int e) {
+  e = max(-126, min(127, e));
+  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
 }
 
-// Row r of a split operand: v holds K2 values; the row is
-// [hi(v), second(v), third(v), 0...] where the thirds are chosen by the caller.
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Writes row r of an fp16 operand with KP columns: v[k] rounded to nearest,
+// zero past K2.
 template <int KP, int K2>
-__device__ __forceinline__ void write_split_row(unsigned char* base, int r, const float (&v)[K2],
-                                                bool a_side) {
-  // element k of the row: part = k / K2 (0, 1, 2), i = k % K2
-  // A side: [hi, hi, lo]; B side: [hi, lo, hi]
+__device__ __forceinline__ void write_row_f16(unsigned char* base, int r, const float (&v)[K2]) {
 #pragma unroll
   for (int k0 = 0; k0 < KP; k0 += 8) {
-    __nv_bfloat16 row[8];
+    uint32_t u[4];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int k = k0 + t;
-      if (k < 3 * K2) {
-        const int part = k / K2, i = k % K2;
-        __nv_bfloat16 hi, lo;
-        split_bf16(v[i], hi, lo);
-        const bool take_lo = a_side ? (part == 2) : (part == 1);
-        row[t] = take_lo ? lo : hi;
-      } else {
-        row[t] = __float2bfloat16_rn(0.f);
-      }
+    for (int t = 0; t < 4; ++t) {
+      const int k = k0 + 2 * t;
+      const float lo = k < K2 ? v[k] : 0.f, hi = k + 1 < K2 ? v[k + 1] : 0.f;
+      const __half2 h2 = __floats2half2_rn(lo, hi);
+      u[t] = *reinterpret_cast<const uint32_t*>(&h2);
     }
-    st_row8(base, op_off<KP>(r, k0), row);
+    *reinterpret_cast<uint4*>(base + op_off<KP>(r, k0)) = make_uint4(u[0], u[1], u[2], u[3]);
   }
+}
+
+// Token n's sub-vector of (group j, head h) and its weights (1 when no
+// weights are given), with one vector load per loop step for each.
+template <int C, int G>
+__device__ __forceinline__ void load_subvector_vec(const EncodeParams& p, int n, int j, int h,
+                                                   float (&s)[C * G], float (&w)[C * G]) {
+#pragma unroll
+  for (int tau = 0; tau < G; ++tau) {
+    const uint16_t* xr = p.x + tau * p.x_loop_stride + n * p.x_token_stride +
+                         static_cast<int64_t>(h) * p.d + j * C;
+    uint32_t u[C / 2];
+    if constexpr (C == 8) {
+      const uint4 t = *reinterpret_cast<const uint4*>(xr);
+      u[0] = t.x; u[1] = t.y; u[2] = t.z; u[3] = t.w;
+    } else if constexpr (C == 4) {
+      const uint2 t = *reinterpret_cast<const uint2*>(xr);
+      u[0] = t.x; u[1] = t.y;
+    } else {
+      u[0] = *reinterpret_cast<const uint32_t*>(xr);
+    }
+#pragma unroll
+    for (int i = 0; i < C / 2; ++i) {
+      s[tau * C + 2 * i] = __uint_as_float(u[i] << 16);
+      s[tau * C + 2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+    if (p.w != nullptr) {
+      const float* wr = p.w + tau * p.w_loop_stride + n * p.w_token_stride +
+                        static_cast<int64_t>(h) * p.d + j * C;
+      if constexpr (C == 2) {
+        const float2 t = *reinterpret_cast<const float2*>(wr);
+        w[tau * C] = t.x; w[tau * C + 1] = t.y;
+      } else {
+#pragma unroll
+        for (int i = 0; i < C; i += 4) {
+          const float4 t = *reinterpret_cast<const float4*>(wr + i);
+          w[tau * C + i] = t.x; w[tau * C + i + 1] = t.y; w[tau * C + i + 2] = t.z; w[tau * C + i + 3] = t.w;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < C; ++ch) w[tau * C + ch] = 1.f;
+    }
+  }
+}
+
+// Byte of (slot, group j, head h) in the pool, or in assign[h][j][slot], for
+// slot < 2^31: one 32-bit division by the block size (page_tokens is a
+// power-of-two multiple of it, and the granule a power of two).
+__device__ __forceinline__ void store_index_u32(const EncodeParams& p, uint32_t slot, int j, int h, int e,
+                                                int pg_shift, int gr_shift) {
+  if (p.assign != nullptr) {
+    p.assign[(static_cast<int64_t>(h) * p.J + j) * p.n_tokens + slot] = static_cast<uint8_t>(e);
+    return;
+  }
+  const uint32_t lb = static_cast<uint32_t>(p.LB), jj = static_cast<uint32_t>(p.J);
+  const uint32_t q = slot / lb;                      // block index over the pool
+  const uint32_t rot = slot - q * lb;                // row in the block
+  const uint32_t page = q >> pg_shift, blk = q & ((1u << pg_shift) - 1u);
+  int pos = j - static_cast<int>(rot % jj);
+  if (pos < 0) pos += p.J;
+  const uint32_t off = blk * lb * jj + ((static_cast<uint32_t>(pos) >> gr_shift) * lb << gr_shift) +
+                       (rot << gr_shift) + (static_cast<uint32_t>(pos) & ((1u << gr_shift) - 1u));
+  p.pool[h * p.pool_stride_head + static_cast<int64_t>(page) * p.page_bytes + p.kv * p.plane_bytes + off] =
+      static_cast<uint8_t>(e);
+}
+
+// 32 consecutive TMEM columns of this warp's 32 lanes, one per register
+// (tcgen05_wait_ld makes them usable).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tcgen05_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 template <int C, int G>
@@ -140,12 +230,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
   unsigned char* Bs = tsm + Geo::B_OFF;
   float* cbs = reinterpret_cast<float*>(tsm + Geo::CB_OFF);
   unsigned int* bmax = reinterpret_cast<unsigned int*>(tsm + Geo::BMAX_OFF);
+  uint32_t* cmask = reinterpret_cast<uint32_t*>(tsm + Geo::MASK_OFF);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(tsm + Geo::MBAR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tsm + Geo::TMEM_OFF);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int j = blockIdx.x, h = blockIdx.y;
 
-  // ---- codebook of (j, h): fp32 copy for rescoring, split B operand -------
+  // ---- codebook of (j, h): fp32 copy for rescoring, scaled fp16 B operand ---
   const float* cb = p.cb + h * p.cb_stride_head + static_cast<int64_t>(j) * kE * C;
   for (int i = tid * 4; i < G * kE * C; i += kTcThreads * 4) {
     const int tau = i / (kE * C), r = i % (kE * C);
@@ -163,8 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
   }
   cp_async_wait_all();
   __syncthreads();
-  for (int e = tid; e < kE; e += kTcThreads) {
-    float b[K2];
+  auto b_row = [&](int e, float (&b)[K2]) {
 #pragma unroll
     for (int tau = 0; tau < G; ++tau) {
 #pragma unroll
@@ -174,31 +264,64 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
         b[D + tau * C + ch] = c * c;
       }
     }
+  };
+  for (int e = tid; e < kE; e += kTcThreads) {
+    float b[K2];
+    b_row(e, b);
 #pragma unroll
     for (int i = 0; i < K2; ++i) atomicMax(bmax + i, __float_as_uint(fabsf(b[i])));
-    write_split_row<KP, K2>(Bs, e, b, false);
+  }
+  __syncthreads();
+  // column scales: the largest |b| of each half lands in [2^13, 2^14)
+  float bm[K2];
+  float m_lo = 0.f, m_hi = 0.f;
+#pragma unroll
+  for (int i = 0; i < K2; ++i) {
+    bm[i] = __uint_as_float(bmax[i]);
+    if (i < D) m_lo = fmaxf(m_lo, bm[i]); else m_hi = fmaxf(m_hi, bm[i]);
+  }
+  const int beta1 = m_lo > 0.f ? kTopExp - exp_of(m_lo) : 0;
+  const int beta2 = m_hi > 0.f ? kTopExp - exp_of(m_hi) : 0;
+  const float fb1 = pow2(beta1), fb2 = pow2(beta2);
+  float q_abs = 0.f;                                 // sum_k max_e |beta'_ek|
+#pragma unroll
+  for (int i = 0; i < K2; ++i) q_abs += bm[i] * (i < D ? fb1 : fb2);
+  // rho keeps 2^rho, 2^(rho - beta1) and 2^(rho - beta2) exact
+  const int rho_lo = max(-126, max(-126 + beta1, -126 + beta2));
+  const int rho_hi = min(127, min(127 + beta1, 127 + beta2));
+  for (int e = tid; e < kE; e += kTcThreads) {
+    float b[K2];
+    b_row(e, b);
+#pragma unroll
+    for (int i = 0; i < K2; ++i) b[i] *= (i < D ? fb1 : fb2);
+    write_row_f16<KP, K2>(Bs, e, b);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // B visible to the tensor cores
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
-  float bm[K2];
-#pragma unroll
-  for (int i = 0; i < K2; ++i) bm[i] = __uint_as_float(bmax[i]);
 
   const uint32_t a_base = u32_smem(As), b_base = u32_smem(Bs), mbar_a = u32_smem(mbar);
   const uint32_t my_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const int n_tiles = (p.n_tokens + kTcRows - 1) / kTcRows;
+  const bool slot_u32 = p.n_slots <= 0x7fffffffLL;
+  const int pg_shift = __ffs(p.Pg / p.LB) - 1, gr_shift = __ffs(p.GR) - 1;
   bool failed = false;
   int last_phase = 0;                                // parity of the MMA commit a failed wait left behind
-  // this thread's token of the next tile, requested one tile ahead
+  // this thread's token of the next tile, requested one tile ahead: its slot
+  // and its data are loaded independently, so neither load waits on the other
   float s_nx[D], w_nx[D];
   int64_t slot_nx = -1;
   auto fetch = [&](int t) {
     const int n = t * kTcRows + tid;
-    slot_nx = (t < n_tiles && n < p.n_tokens) ? token_slot(p, n) : -1;
-    if (slot_nx >= 0 && slot_nx < p.n_slots) load_subvector<C, G>(p, n, j, h, s_nx, w_nx);
+    if (t < n_tiles && n < p.n_tokens) {
+      // the slot's range check waits for the load, so it is made at use
+      slot_nx = p.slot_mapping != nullptr ? p.slot_mapping[n] : static_cast<int64_t>(n);
+      load_subvector_vec<C, G>(p, n, j, h, s_nx, w_nx);
+    } else {
+      slot_nx = -1;
+    }
   };
   fetch(0);
   for (int t = 0; t < n_tiles; ++t) {
@@ -212,28 +335,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
     }
     float a[K2];
     float margin = 0.f;
+    if (slot >= p.n_slots && p.status != nullptr) atomicOr(p.status, LOOPVQ_ENCODE_STATUS_BAD_SLOT);
     const bool live = slot >= 0 && slot < p.n_slots;
     if (live) {
-      float ms = 0.f, wss = 0.f;
+      float m1 = 0.f, m2 = 0.f, wss = 0.f, pu = 0.f;
 #pragma unroll
       for (int i = 0; i < D; ++i) {
         a[i] = w[i] * s[i];
         a[D + i] = w[i];
-        wss = fmaf(w[i] * s[i], s[i], wss);
+        m1 = fmaxf(m1, fabsf(a[i]));
+        m2 = fmaxf(m2, fabsf(w[i]));
+        wss = fmaf(a[i], s[i], wss);
       }
 #pragma unroll
-      for (int i = 0; i < K2; ++i) ms = fmaf(fabsf(a[i]), bm[i], ms);
-      margin = ldexpf(ms + wss, -12);
+      for (int i = 0; i < K2; ++i) pu = fmaf(fabsf(a[i]), bm[i], pu);
+      const int e1 = m1 > 0.f ? exp_of(m1) - beta1 : -100000;
+      const int e2 = m2 > 0.f ? exp_of(m2) - beta2 : -100000;
+      const int er = max(e1, e2);
+      const int rho = max(rho_lo, min(rho_hi, er == -100000 ? 0 : kTopExp - er));
+      const float f1 = pow2(rho - beta1), f2 = pow2(rho - beta2), fr = pow2(rho);
+      float sa = 0.f;
+#pragma unroll
+      for (int i = 0; i < D; ++i) {
+        a[i] *= f1;
+        a[D + i] *= f2;
+        sa += fabsf(a[i]) + fabsf(a[D + i]);
+      }
+      margin = fr * fmaf(kMarginRel, pu, kMarginWss * wss) + kMarginAbs * (sa + q_abs);
+      if (rho_lo > rho_hi) margin = INFINITY;      // no exact scaling: rescore everything
     } else {
 #pragma unroll
       for (int i = 0; i < K2; ++i) a[i] = 0.f;
     }
-    write_split_row<KP, K2>(As, tid, a, true);
+    write_row_f16<KP, K2>(As, tid, a);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
 
-    // ---- S = A . B^T into tensor memory ----------------------------------------
+    // ---- S' = A . B^T into tensor memory ---------------------------------------
     if (tid == 0) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll
@@ -265,65 +404,72 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const EncodePa
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
     // ---- this row's minimum, then the exact rescore within the margin ----------
-    float smin = INFINITY;
+    float m0 = INFINITY, mA = INFINITY, mB = INFINITY, mC = INFINITY;
 #pragma unroll 1
-    for (int c0 = 0; c0 < kE; c0 += 32) {
-      uint32_t r[32];
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-          "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-          "%30, %31}, [%32];"
-          : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-            "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-            "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-            "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-            "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-          : "r"(my_tmem + c0));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    for (int c0 = 0; c0 < kE; c0 += 64) {
+      uint32_t r[32], r2[32];
+      tmem_ld32_async(my_tmem + c0, r);
+      tmem_ld32_async(my_tmem + c0 + 32, r2);
+      tcgen05_wait_ld();
 #pragma unroll
-      for (int q = 0; q < 32; ++q) smin = fminf(smin, __uint_as_float(r[q]));
-    }
-    const float thr = smin + margin;
-    float best = INFINITY;
-    int best_e = 0;
-#pragma unroll 1
-    for (int c0 = 0; c0 < kE; c0 += 32) {
-      uint32_t r[32];
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-          "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-          "%30, %31}, [%32];"
-          : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-            "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-            "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-            "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-            "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-          : "r"(my_tmem + c0));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      if (!live) continue;
-      uint32_t cand = 0u;                            // columns within the margin, ascending
-#pragma unroll
-      for (int q = 0; q < 32; ++q) cand |= (__uint_as_float(r[q]) <= thr ? 1u : 0u) << q;
-      while (cand != 0u) {
-        const int e = c0 + __ffs(cand) - 1;
-        cand &= cand - 1u;
-        float dist = 0.f;                            // encode_kernel's terms, in its order
-#pragma unroll
-        for (int tau = 0; tau < G; ++tau) {
-          const float* cw = cbs + (tau * kE + e) * C;
-#pragma unroll
-          for (int ch = 0; ch < C; ++ch) {
-            const float df = s[tau * C + ch] - cw[ch];
-            dist = fmaf(w[tau * C + ch] * df, df, dist);
-          }
-        }
-        if (dist < best) {
-          best = dist;
-          best_e = e;
-        }
+      for (int q = 0; q < 32; q += 4) {
+        m0 = min3f(m0, __uint_as_float(r[q]), __uint_as_float(r[q + 1]));
+        mA = min3f(mA, __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
+        mB = min3f(mB, __uint_as_float(r2[q]), __uint_as_float(r2[q + 1]));
+        mC = min3f(mC, __uint_as_float(r2[q + 2]), __uint_as_float(r2[q + 3]));
       }
     }
-    if (live) store_index(p, slot, j, h, best_e);
+    const float smin = fminf(min3f(m0, mA, mB), mC);
+    float thr = smin + margin;
+    if (!(fabsf(smin) < INFINITY) || !(margin < INFINITY)) thr = INFINITY;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kE; c0 += 64) {
+      uint32_t r[32], r2[32];
+      tmem_ld32_async(my_tmem + c0, r);
+      tmem_ld32_async(my_tmem + c0 + 32, r2);
+      tcgen05_wait_ld();
+      uint32_t cand = 0u, cand2 = 0u;                // columns within the margin, ascending
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        cand |= (__uint_as_float(r[q]) > thr ? 0u : 1u) << q;
+        cand2 |= (__uint_as_float(r2[q]) > thr ? 0u : 1u) << q;
+      }
+      cmask[(c0 >> 5) * kTcRows + tid] = live ? cand : 0u;
+      cmask[((c0 >> 5) + 1) * kTcRows + tid] = live ? cand2 : 0u;
+    }
+    // every candidate of the row in one loop, in ascending order, so that a
+    // warp runs as many rescoring rounds as its busiest lane has candidates
+    float best = INFINITY;
+    int best_e = 0;
+    int chunk = 0;
+    uint32_t m = cmask[tid];
+#pragma unroll 1
+    for (;;) {
+      while (m == 0u && chunk < kE / 32 - 1) m = cmask[++chunk * kTcRows + tid];
+      if (m == 0u) break;
+      const int e = chunk * 32 + __ffs(m) - 1;
+      m &= m - 1u;
+      float dist = 0.f;                              // encode_kernel's terms, in its order
+#pragma unroll
+      for (int tau = 0; tau < G; ++tau) {
+        const float* cw = cbs + (tau * kE + e) * C;
+#pragma unroll
+        for (int ch = 0; ch < C; ++ch) {
+          const float df = s[tau * C + ch] - cw[ch];
+          dist = fmaf(w[tau * C + ch] * df, df, dist);
+        }
+      }
+      if (dist < best) {
+        best = dist;
+        best_e = e;
+      }
+    }
+    if (live) {
+      if (slot_u32)
+        store_index_u32(p, static_cast<uint32_t>(slot), j, h, best_e, pg_shift, gr_shift);
+      else
+        store_index(p, slot, j, h, best_e);
+    }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();                                 // TMEM read, A free for the next tile
   }
