@@ -162,8 +162,10 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
 
 template <int C, int G>
 loopvq_status launch_enc(const EncodeParams& p, int J, int H, cudaStream_t st) {
-  if (p.n_tokens >= kEncTcMinTokens && encode_tc_supported(C, G))
-    return launch_encode_tc(p, C, G, J, H, st);
+  if (p.n_tokens >= kEncTcMinTokens && encode_tc_supported(C, G)) {
+    const loopvq_status r = launch_encode_tc(p, C, G, J, H, st);
+    if (r != LOOPVQ_ERR_UNSUPPORTED) return r;       // else: inputs TMA cannot describe, direct form
+  }
   if (p.n_tokens <= kEncWarpMaxTokens) {
     encode_warp_kernel<C, G><<<dim3(J, H), kEncWarpThreads, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
