@@ -80,7 +80,14 @@ enum {
   /* a range check of a build with LOOPVQ_RANGE_CHECK defined found an index
    * outside its buffer; the access was skipped (never set by the default
    * build, whose indices are in range by construction) */
-  LOOPVQ_DECODE_STATUS_RANGE = 4
+  LOOPVQ_DECODE_STATUS_RANGE = 4,
+  /* a bounded wait of the tensor-core prefill form (for the tensor cores or
+   * a bulk copy) gave up; the affected records are NaN and the call's
+   * outputs are not to be trusted */
+  LOOPVQ_DECODE_STATUS_TIMEOUT = 8,
+  /* with LOOPVQ_DECODE_STATUS_TIMEOUT: the work in flight could not be
+   * waited for before the kernel exited */
+  LOOPVQ_DECODE_STATUS_UNDRAINED = 16
 };
 
 /*

@@ -11,6 +11,8 @@ from .binding import (  # noqa: F401
     LOOPVQ_ENCODE_STATUS_BAD_SLOT,
     LOOPVQ_DECODE_STATUS_RANGE,
     LOOPVQ_DECODE_STATUS_SHARED_BASE,
+    LOOPVQ_DECODE_STATUS_TIMEOUT,
+    LOOPVQ_DECODE_STATUS_UNDRAINED,
     LOOPVQ_DTYPE_BF16,
     LOOPVQ_DTYPE_F32,
     LoopVQConfig,

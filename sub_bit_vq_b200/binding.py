@@ -33,6 +33,8 @@ LOOPVQ_ENCODE_STATUS_BAD_SLOT = 4
 LOOPVQ_DECODE_STATUS_BAD_PAGE = 1
 LOOPVQ_DECODE_STATUS_SHARED_BASE = 2
 LOOPVQ_DECODE_STATUS_RANGE = 4
+LOOPVQ_DECODE_STATUS_TIMEOUT = 8
+LOOPVQ_DECODE_STATUS_UNDRAINED = 16
 
 
 class LoopVQError(RuntimeError):

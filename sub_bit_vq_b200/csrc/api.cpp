@@ -303,6 +303,10 @@ loopvq_status decode_common(const loopvq_config* cfg, int layer, int loop_step, 
   DecodeArgs a{&g,        layer,       loop_step, batch, n_queries, max_seq_len, q,        pool,
                codebooks, block_table, seq_lens,  win_k, win_v,     sm_scale,    out_dtype, out,
                lse,       workspace,   n_cta,     stream};
+  if (prefill_tc_supported(g, n_queries, out_dtype)) {
+    const loopvq_status r = launch_prefill_tc(a, workspace_bytes);
+    if (r != LOOPVQ_ERR_UNSUPPORTED) return r;     // else the streaming form below
+  }
   return launch_decode(a);
 }
 

@@ -63,6 +63,18 @@ struct DecodeArgs {
 };
 loopvq_status launch_decode(const DecodeArgs& a);
 
+// The tensor-core form of attention over the cache for chunks of at least
+// kPrefillTcMinQueries queries per sequence (prefill_tc.cu): bf16 outputs,
+// head_dim 128 at c = 4. It keeps split records of (d + 2) floats per
+// query row and token chunk, and the key and value codebook slices in bf16,
+// in the workspace; when `workspace_bytes` cannot hold them it returns
+// LOOPVQ_ERR_UNSUPPORTED and launches nothing.
+constexpr int kPrefillTcMinQueries = 64;
+bool prefill_tc_supported(const Geometry& g, int n_queries, int out_dtype);
+size_t prefill_tc_workspace_bytes(const Geometry& g, int batch, int n_queries, int max_seq_len, int* S,
+                                  int* CH);
+loopvq_status launch_prefill_tc(const DecodeArgs& a, size_t workspace_bytes);
+
 struct EncodeArgs {
   const Geometry* geo;
   int layer, gamma, kv, n_tokens;

@@ -217,7 +217,8 @@ def test_status_bits_match_the_header():
     text = open(os.path.join(ROOT, "include", "loopvq.h")).read()
     for name in ("LOOPVQ_DECODE_STATUS_BAD_PAGE", "LOOPVQ_DECODE_STATUS_SHARED_BASE",
                  "LOOPVQ_ENCODE_STATUS_TIMEOUT", "LOOPVQ_ENCODE_STATUS_UNDRAINED",
-                 "LOOPVQ_ENCODE_STATUS_BAD_SLOT", "LOOPVQ_DECODE_STATUS_RANGE"):
+                 "LOOPVQ_ENCODE_STATUS_BAD_SLOT", "LOOPVQ_DECODE_STATUS_RANGE",
+                 "LOOPVQ_DECODE_STATUS_TIMEOUT", "LOOPVQ_DECODE_STATUS_UNDRAINED"):
         m = re.search(name + r"\s*=\s*(\d+)", text)
         assert m, name
         assert getattr(B, name) == int(m.group(1)) == getattr(L, name)
