@@ -11,12 +11,14 @@
 //
 // Work unit: (sequence b, query head hq, tile of 128 queries, token chunk).
 // Chunks 0 .. S-2 cover the quantised tokens [c*CH, (c+1)*CH); chunk S-1 is
-// the bf16 window (prefix + recent). One CTA (128 threads, thread r = query
-// row r = TMEM lane r) per unit:
+// the bf16 window (prefix + recent). One CTA per unit, 256 threads: query
+// row r (TMEM lane r) is served by a thread of warp r / 32 and one of warp
+// r / 32 + 4, each holding half of the row's S, P and O columns:
 //   1. Q tile (bf16, K-major, no swizzle) into shared memory; the (layer,
-//      kv-head, gamma, tau) key codebook slice (fp32, 128 KB) by bulk copy
-//      into shared memory. The value slice, rounded to bf16 by
-//      prefill_cb_kernel, stays in global memory (L2) and is gathered.
+//      kv-head, gamma, tau) key codebook slice, split by prefill_cb_kernel
+//      into bf16 high and low parts (128 KB), by bulk copy into shared
+//      memory. The value slice, rounded to bf16, stays in global memory (L2)
+//      and is gathered.
 //   2. Per tile of 64 tokens: the key indices of the tile (rotated rows of the
 //      pool's K plane) select codewords, split into bf16 high and low parts,
 //      into K_hi and K_lo [64][d]; the value indices select bf16 codewords
@@ -48,7 +50,7 @@ namespace {
 
 constexpr int kPfRows = 128;              // queries per tile (MMA M)
 constexpr int kPfTok = 64;                // tokens per tile
-constexpr int kPfThreads = 128;
+constexpr int kPfThreads = 256;            // two threads per query row (column halves)
 constexpr int kPfD = 128;                 // head_dim of this form
 constexpr int kPfJ = 32;                  // channel groups (c = 4)
 constexpr int kPfC = 4;
@@ -78,8 +80,7 @@ struct PrefillParams {
   const uint16_t* q;              // bf16 [B][Q][Hq][d]
   const uint8_t* pool_lg;         // pool at (layer, gamma, head 0)
   int64_t pool_stride_head, page_bytes, plane_bytes;
-  const float* cb_k;              // key slices at (layer, head 0, gamma, tau): [J][E][C] fp32
-  int64_t cb_stride_head;
+  const uint16_t* cbk16;          // bf16 key slices split high/low [Hkv][J][E][2][C]
   const uint16_t* cbv16;          // bf16 value slices [Hkv][J][E][C]
   const int32_t* block_table;
   const int32_t* seq_lens;
@@ -169,16 +170,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// The value codebook slices of every kv-head at loop offset tau, rounded to
-// bf16: cbv16[h][j][e][ch].
-__global__ void __launch_bounds__(256) prefill_cb_kernel(const float* cb_v, int64_t cb_stride_head, int Hkv,
-                                                         uint16_t* cbv16) {
+// The codebook slices of every kv-head at loop offset tau in bf16: the value
+// slice rounded, cbv16[h][j][e][ch], and the key slice split into high and
+// low parts, cbk16[h][j][e][hi 0..3, lo 0..3] (16 bytes per codeword).
+__global__ void __launch_bounds__(256) prefill_cb_kernel(const float* cb_k, const float* cb_v,
+                                                         int64_t cb_stride_head, int Hkv, uint16_t* cbv16,
+                                                         uint16_t* cbk16) {
   constexpr int N = kCb16Elems;
   const int64_t total = static_cast<int64_t>(Hkv) * N;
   for (int64_t i = (blockIdx.x * 256 + threadIdx.x) * 4ll; i < total; i += gridDim.x * 256ll * 4) {
     const int h = static_cast<int>(i / N), r = static_cast<int>(i % N);
     const float4 v = *reinterpret_cast<const float4*>(cb_v + h * cb_stride_head + r);
     *reinterpret_cast<uint2*>(cbv16 + i) = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+    const float4 k = *reinterpret_cast<const float4*>(cb_k + h * cb_stride_head + r);
+    const __nv_bfloat162 h01 = __floats2bfloat162_rn(k.x, k.y), h23 = __floats2bfloat162_rn(k.z, k.w);
+    const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+    const __nv_bfloat162 l01 = __floats2bfloat162_rn(k.x - f01.x, k.y - f01.y);
+    const __nv_bfloat162 l23 = __floats2bfloat162_rn(k.z - f23.x, k.w - f23.y);
+    *reinterpret_cast<uint4*>(cbk16 + 2 * i) =
+        make_uint4(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23),
+                   *reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
   }
 }
 
@@ -188,11 +199,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
   unsigned char* Ks = sm + kKsOff;
   unsigned char* Vs = sm + kVsOff;
   unsigned char* Ps = sm + kPsOff;
-  const float* cbk = reinterpret_cast<const float*>(sm + kCbOff);
+  const uint4* cbk = reinterpret_cast<const uint4*>(sm + kCbOff);   // [J][E] (hi, lo) codewords
   uint8_t* vix = sm + kVixOff;
+  float* xch = reinterpret_cast<float*>(sm + kVixOff);   // [2][128] row partials (vix is free then)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kTmemOff);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = ((warp & 3) << 5) | lane;            // query row of the tile = TMEM lane
+  const int colh = warp >> 2;                          // half of the S, P and O columns
 
   // ---- the unit -----------------------------------------------------------------
   int x = blockIdx.x;
@@ -207,19 +221,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
   const bool window = c == p.S - 1;
   const int k0 = window ? 0 : c * p.CH;
   const int k1 = window ? min(N, p.W) : min(n_vq, (c + 1) * p.CH);   // tokens [k0, k1)
-  const int row_q = qt * kPfRows + tid;                // this thread's query
+  const int row_q = qt * kPfRows + row;                // this thread's query
   const bool row_ok = row_q < p.Q;
   float* rec = p.records + ((static_cast<size_t>(b) * p.Q + row_q) * p.Hq + hq) * p.S * (kPfD + 2) +
                static_cast<size_t>(c) * (kPfD + 2);
   if (k1 <= k0) {                                      // CTA-uniform: an empty record
-    if (row_ok) {
+    if (row_ok && colh == 0) {
       rec[0] = -INFINITY;
       rec[1] = 0.f;
     }
     return;
   }
 
-  // ---- setup: barriers, TMEM, codebooks, Q tile ------------------------------------
+  // ---- setup: barriers, TMEM, key codebook, Q tile ---------------------------------
   const uint32_t bar_s = u32s(bars), bar_o = u32s(bars + 1), bar_cb = u32s(bars + 2);
   if (tid == 0) {
     for (int i = 0; i < 3; ++i)
@@ -235,25 +249,26 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
   if (tid == 0 && !window) {                           // the key slice: two bulk copies of 64 KB
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_cb), "r"(kCbBytes)
                  : "memory");
-    const float* src = p.cb_k + hkv * p.cb_stride_head;
+    const uint16_t* src = p.cbk16 + static_cast<size_t>(hkv) * (kCbBytes / 2);
     for (int part = 0; part < 2; ++part)
       asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                   ::"r"(u32s(sm + kCbOff + part * (kCbBytes / 2))), "l"(src + part * (kCbBytes / 8)),
+                   ::"r"(u32s(sm + kCbOff + part * (kCbBytes / 2))), "l"(src + part * (kCbBytes / 4)),
                    "r"(kCbBytes / 2), "r"(bar_cb) : "memory");
   }
   {                                                    // the query rows, bf16, zero past Q
-    const uint16_t* qr = p.q + ((static_cast<size_t>(b) * p.Q + row_q) * p.Hq + hq) * kPfD;
-#pragma unroll 4
-    for (int k0c = 0; k0c < kPfD; k0c += 8) {
-      const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qr + k0c) : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(Qs + kmaj<kPfD>(tid, k0c)) = v;
+    const uint16_t* qr = p.q + ((static_cast<size_t>(b) * p.Q + row_q) * p.Hq + hq) * kPfD + colh * 64;
+#pragma unroll
+    for (int k = 0; k < 64; k += 8) {
+      const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qr + k) : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(Qs + kmaj<kPfD>(row, colh * 64 + k)) = v;
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+  const uint32_t my_s = lane_base + kTmemS + colh * 32, my_o = lane_base + kTmemO + colh * 64;
   bool failed = !window && !pf_wait(bar_cb, 0, kPfSpin);
   failed = __syncthreads_or(failed);
 
@@ -263,14 +278,102 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
   const uint16_t* wv = p.win_v + (static_cast<size_t>(b) * (p.Hq / p.ratio) + hkv) * p.W * kPfD;
   const uint32_t qs_a = u32s(Qs), ks_a = u32s(Ks), vs_a = u32s(Vs), ps_a = u32s(Ps);
   const uint16_t* cbv = p.cbv16 + static_cast<size_t>(hkv) * kCb16Elems;   // bf16, in L2
-  float m_run = -INFINITY, l_run = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;                // l_run: this thread's half of the row
   bool o_live = false;                                 // an O product has been issued
   int n_tiles_done = 0;
   int pending_o = -1;                                  // parity of an O commit not yet waited for
 
+  // Index bytes of this thread's token (t & 63) and quarter (t >> 6) of the
+  // tile at token tt, requested one tile ahead; its page entry two tiles ahead.
+  uint2 nx_k = make_uint2(0u, 0u), nx_v = make_uint2(0u, 0u);
+  bool nx_ok = false;
+  int ph_a = -1, ph_b = -1;                            // page entries of my token in the next two tiles
+  auto page_of = [&](int tt) -> int {                  // block-table entry of my token at tile tt
+    const int kq = tt + (tid & 63);
+    return (tt < k1 && kq < k1) ? bt[kq / p.Pg] : -1;
+  };
+  auto fetch_rows = [&](int tt) {                      // rows of tile tt (page entry ph_a); shift the entries
+    const int kq = tt + (tid & 63), quarter = tid >> 6;
+    const bool tok = tt < k1 && kq < k1;
+    nx_ok = tok && ph_a >= 0 && ph_a < p.n_pages;
+    if (tok && !nx_ok && quarter == 0 && p.status != nullptr) atomicOr(p.status, LOOPVQ_DECODE_STATUS_BAD_PAGE);
+    nx_k = make_uint2(0u, 0u);
+    nx_v = make_uint2(0u, 0u);
+    if (nx_ok) {
+      const int slot = kq % p.Pg, blk = slot / p.LB, rot = slot % p.LB;
+      const uint8_t* rowp = pool_h + static_cast<int64_t>(ph_a) * p.page_bytes + blk * (p.LB * kPfJ) +
+                            (quarter >> 1) * (p.LB * 16) + rot * 16 + (quarter & 1) * 8;
+      nx_k = *reinterpret_cast<const uint2*>(rowp);
+      nx_v = *reinterpret_cast<const uint2*>(rowp + p.plane_bytes);
+    }
+    ph_a = ph_b;
+    ph_b = page_of(tt + 2 * kPfTok);
+  };
+  if (!window) {
+    ph_a = page_of(k0);
+    ph_b = page_of(k0 + kPfTok);
+    fetch_rows(k0);                                    // tile 0 now, entries of tiles 1 and 2 in flight
+  }
+
   for (int t0 = k0; t0 < k1 && !failed; t0 += kPfTok) {
     const int nt = min(kPfTok, k1 - t0);               // valid tokens of this tile
-    // the previous tile's O product has read Ps and Vs
+
+    // ---- index bytes of this tile (prefetched a tile ago) and the next tile's ---------
+    const int n = tid & 63, quarter = tid >> 6;        // token of the tile, quarter of its 32 groups
+    const bool tok_ok = n < nt;
+    uint2 kidx = make_uint2(0u, 0u);
+    bool page_ok = false;
+    if (!window) {
+      kidx = nx_k;
+      page_ok = nx_ok;
+      *reinterpret_cast<uint2*>(vix + n * kPfJ + quarter * 8) = nx_v;   // value bytes by position
+      fetch_rows(t0 + kPfTok);                         // tile t + 1: lands during this tile
+    }
+    if (!window) __syncthreads();                      // value index bytes staged
+    // ---- value codewords of this tile: task (group j, token octet o) gathers dims
+    // 4j .. 4j+3 of tokens 8o .. 8o+7 (from L2; they land while K is dequantised)
+    const int vj = tid & (kPfJ - 1), vo = tid >> 5;
+    uint32_t vlo[8], vhi[8];                           // token q: dims (4j, 4j+1) and (4j+2, 4j+3)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int tn = vo * 8 + q;
+      uint2 cw = make_uint2(0u, 0u);
+      if (tn < nt) {
+        if (window) {
+          cw = *reinterpret_cast<const uint2*>(wv + static_cast<size_t>(t0 + tn) * kPfD + vj * kPfC);
+        } else {
+          const int rot = ((t0 + tn) % p.Pg) % p.LB;
+          const int pos = (vj - rot) & (kPfJ - 1);
+          const uint32_t idx = vix[tn * kPfJ + pos];
+          cw = *reinterpret_cast<const uint2*>(cbv + (vj * kE + idx) * kPfC);
+        }
+      }
+      vlo[q] = cw.x;
+      vhi[q] = cw.y;
+    }
+    // ---- K tile [64][128] (hi, lo); the previous S product is done with Ks ------------
+    if (window) {
+      const uint16_t* kr = wk + static_cast<size_t>(t0 + n) * kPfD + quarter * 32;
+#pragma unroll
+      for (int k = 0; k < 32; k += 8) {
+        const uint4 v = tok_ok ? *reinterpret_cast<const uint4*>(kr + k) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(Ks + kmaj<kPfD>(n, quarter * 32 + k)) = v;               // exact in bf16
+        *reinterpret_cast<uint4*>(Ks + kKsBytes + kmaj<kPfD>(n, quarter * 32 + k)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else {
+      const int rot = ((t0 + n) % p.Pg) % p.LB;
+      const uint32_t kw[2] = {kidx.x, kidx.y};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int pos = quarter * 8 + q;
+        const int j = (pos + rot) & (kPfJ - 1);        // group of this byte of the rotated row
+        const uint32_t idx = (kw[q >> 2] >> (8 * (q & 3))) & 0xffu;
+        const uint4 cw = page_ok ? cbk[j * kE + idx] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint2*>(Ks + kmaj<kPfD>(n, j * kPfC)) = make_uint2(cw.x, cw.y);
+        *reinterpret_cast<uint2*>(Ks + kKsBytes + kmaj<kPfD>(n, j * kPfC)) = make_uint2(cw.z, cw.w);
+      }
+    }
+    // the previous tile's O product has read Ps and Vs (and O may be rescaled)
     if (pending_o >= 0) {
       const bool ok = pf_wait(bar_o, static_cast<uint32_t>(pending_o), kPfSpin);
       if (__syncthreads_or(!ok)) {
@@ -280,100 +383,22 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
       pending_o = -1;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     }
-
-    // ---- K tile [64][128] and V^T tile [128][64] ---------------------------------
-    {
-      const int n = tid & 63, half = tid >> 6;         // token of the tile, half of its 32 groups
-      const bool tok_ok = n < nt;
-      if (window) {
-        // bf16 window tokens: the K row directly, the V row transposed below
-        const uint16_t* kr = wk + static_cast<size_t>(t0 + n) * kPfD + half * 64;
 #pragma unroll
-        for (int k = 0; k < 64; k += 8) {
-          const uint4 v = tok_ok ? *reinterpret_cast<const uint4*>(kr + k) : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(Ks + kmaj<kPfD>(n, half * 64 + k)) = v;              // exact in bf16
-          *reinterpret_cast<uint4*>(Ks + kKsBytes + kmaj<kPfD>(n, half * 64 + k)) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      } else {
-        // quantised token t0 + n: page, slot, rotated row; granule `half` of
-        // its K row holds positions 16 half .. 16 half + 15
-        const int kq = t0 + n;
-        const int pg = kq / p.Pg, slot = kq % p.Pg;
-        const int phys = tok_ok ? bt[pg] : -1;
-        const bool page_ok = tok_ok && phys >= 0 && phys < p.n_pages;
-        if (tok_ok && !page_ok && half == 0 && p.status != nullptr) atomicOr(p.status, LOOPVQ_DECODE_STATUS_BAD_PAGE);
-        const int blk = slot / p.LB, rot = slot % p.LB;
-        uint4 kidx = make_uint4(0u, 0u, 0u, 0u), vidx = make_uint4(0u, 0u, 0u, 0u);
-        if (page_ok) {
-          const uint8_t* row = pool_h + static_cast<int64_t>(phys) * p.page_bytes + blk * (p.LB * kPfJ) +
-                               half * (p.LB * 16) + rot * 16;
-          kidx = *reinterpret_cast<const uint4*>(row);
-          vidx = *reinterpret_cast<const uint4*>(row + p.plane_bytes);
-        }
-        *reinterpret_cast<uint4*>(vix + n * kPfJ + half * 16) = vidx;   // value bytes by position
-        const uint32_t kw[4] = {kidx.x, kidx.y, kidx.z, kidx.w};
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int pos = half * 16 + q;
-          const int j = (pos + rot) & (kPfJ - 1);      // group of this byte of the rotated row
-          const uint32_t idx = (kw[q >> 2] >> (8 * (q & 3))) & 0xffu;
-          const float4 cw = page_ok ? *reinterpret_cast<const float4*>(cbk + (j * kE + idx) * kPfC)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-          const __nv_bfloat162 h01 = __floats2bfloat162_rn(cw.x, cw.y), h23 = __floats2bfloat162_rn(cw.z, cw.w);
-          const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-          const __nv_bfloat162 l01 = __floats2bfloat162_rn(cw.x - f01.x, cw.y - f01.y);
-          const __nv_bfloat162 l23 = __floats2bfloat162_rn(cw.z - f23.x, cw.w - f23.y);
-          *reinterpret_cast<uint2*>(Ks + kmaj<kPfD>(n, j * kPfC)) =
-              make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
-          *reinterpret_cast<uint2*>(Ks + kKsBytes + kmaj<kPfD>(n, j * kPfC)) =
-              make_uint2(*reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
-        }
-      }
-    }
-    if (!window) __syncthreads();                      // value index bytes staged
-    {
-      // V^T: task (group j, token octet o) writes dims 4j .. 4j+3 of tokens 8o .. 8o+7
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int task = tid + rr * kPfThreads;
-        const int j = task & (kPfJ - 1), o = task >> 5;
-        uint32_t lo[8], hi[8];                         // token q: dims (4j, 4j+1) and (4j+2, 4j+3)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int n = o * 8 + q;
-          uint2 cw = make_uint2(0u, 0u);
-          if (n < nt) {
-            if (window) {
-              cw = *reinterpret_cast<const uint2*>(wv + static_cast<size_t>(t0 + n) * kPfD + j * kPfC);
-            } else {
-              const int rot = ((t0 + n) % p.Pg) % p.LB;
-              const int pos = (j - rot) & (kPfJ - 1);
-              const uint32_t idx = vix[n * kPfJ + pos];
-              cw = *reinterpret_cast<const uint2*>(cbv + (j * kE + idx) * kPfC);
-            }
-          }
-          lo[q] = cw.x;
-          hi[q] = cw.y;
-        }
-        // dim 4j + ch: 8 tokens, 16 bytes
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const uint32_t* src = ch < 2 ? lo : hi;
-          const uint32_t sel = (ch & 1) ? 0x7632u : 0x5410u;   // high or low bf16 of each word
-          uint4 v;
-          v.x = __byte_perm(src[0], src[1], sel);
-          v.y = __byte_perm(src[2], src[3], sel);
-          v.z = __byte_perm(src[4], src[5], sel);
-          v.w = __byte_perm(src[6], src[7], sel);
-          *reinterpret_cast<uint4*>(Vs + kmaj<kPfTok>(4 * j + ch, o * 8)) = v;
-        }
-      }
+    for (int ch = 0; ch < 4; ++ch) {                   // V^T row 4j + ch: 8 tokens, 16 bytes
+      const uint32_t* src = ch < 2 ? vlo : vhi;
+      const uint32_t sel = (ch & 1) ? 0x7632u : 0x5410u;   // high or low bf16 of each word
+      uint4 v;
+      v.x = __byte_perm(src[0], src[1], sel);
+      v.y = __byte_perm(src[2], src[3], sel);
+      v.z = __byte_perm(src[4], src[5], sel);
+      v.w = __byte_perm(src[6], src[7], sel);
+      *reinterpret_cast<uint4*>(Vs + kmaj<kPfTok>(4 * vj + ch, vo * 8)) = v;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
 
-    // ---- S = Q K^T ------------------------------------------------------------------
+    // ---- S = Q K_hi^T + Q K_lo^T -------------------------------------------------------
     const int tile = n_tiles_done;
     if (tid == 0) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -395,33 +420,33 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
     }
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
-    // ---- softmax of this row; P into shared memory ------------------------------------
-    uint32_t s0[32], s1[32];
-    tld32(lane_base + kTmemS, s0);
-    tld32(lane_base + kTmemS + 32, s1);
+    // ---- softmax: this thread's 32 columns of its row; P into shared memory ------------
+    uint32_t sv[32];
+    tld32(my_s, sv);
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
     float mt = -INFINITY;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float a0 = i < nt ? __uint_as_float(s0[i]) * p.scale_log2 : -INFINITY;
-      const float a1 = 32 + i < nt ? __uint_as_float(s1[i]) * p.scale_log2 : -INFINITY;
-      s0[i] = __float_as_uint(a0);
-      s1[i] = __float_as_uint(a1);
-      mt = fmaxf(mt, fmaxf(a0, a1));
+      const float a = colh * 32 + i < nt ? __uint_as_float(sv[i]) * p.scale_log2 : -INFINITY;
+      sv[i] = __float_as_uint(a);
+      mt = fmaxf(mt, a);
     }
+    xch[colh * kPfRows + row] = mt;
+    __syncthreads();
+    mt = fmaxf(xch[row], xch[kPfRows + row]);          // the row's maximum over both halves
     const bool raise = m_run == -INFINITY || mt > m_run + kPfLazy;
-    if (__any_sync(0xffffffffu, raise)) {              // warp-uniform: rescale this warp's rows
+    if (__any_sync(0xffffffffu, raise)) {              // warp-uniform; the partner warp decides alike
       const float m_new = raise ? fmaxf(m_run, mt) : m_run;
       const float alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
       if (o_live) {
 #pragma unroll 1
-        for (int cc = 0; cc < kPfD; cc += 32) {
+        for (int cc = 0; cc < 64; cc += 32) {
           uint32_t o[32];
-          tld32(lane_base + kTmemO + cc, o);
+          tld32(my_o + cc, o);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tst32(lane_base + kTmemO + cc, o);
+          tst32(my_o + cc, o);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
@@ -429,19 +454,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
       m_run = m_new;
     }
 #pragma unroll
-    for (int k = 0; k < kPfTok; k += 8) {
+    for (int k = 0; k < 32; k += 8) {
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int i0 = k + 2 * e;
-        const float x0 = __uint_as_float(i0 < 32 ? s0[i0] : s1[i0 - 32]);
-        const float x1 = __uint_as_float(i0 + 1 < 32 ? s0[i0 + 1] : s1[i0 + 1 - 32]);
-        const float p0 = fast_exp2(x0 - m_run), p1 = fast_exp2(x1 - m_run);
+        const float p0 = fast_exp2(__uint_as_float(sv[k + 2 * e]) - m_run);
+        const float p1 = fast_exp2(__uint_as_float(sv[k + 2 * e + 1]) - m_run);
         l_run += p0 + p1;                              // unrounded: lse keeps float32 precision
         const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
         w[e] = *reinterpret_cast<const uint32_t*>(&pb);
       }
-      *reinterpret_cast<uint4*>(Ps + kmaj<kPfTok>(tid, k)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(Ps + kmaj<kPfTok>(row, colh * 32 + k)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -470,19 +493,22 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
   if (!failed) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll 1
-    for (int cc = 0; cc < kPfD; cc += 32) {
+    for (int cc = 0; cc < 64; cc += 32) {
       uint32_t o[32];
-      tld32(lane_base + kTmemO + cc, o);
+      tld32(my_o + cc, o);
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       if (row_ok) {
 #pragma unroll
         for (int i = 0; i < 32; i += 2)                // records are 8-byte aligned
-          *reinterpret_cast<float2*>(rec + 2 + cc + i) = make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1]));
+          *reinterpret_cast<float2*>(rec + 2 + colh * 64 + cc + i) =
+              make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1]));
       }
     }
-    if (row_ok) {
+    xch[colh * kPfRows + row] = l_run;
+    __syncthreads();
+    if (row_ok && colh == 0) {
       rec[0] = m_run;
-      rec[1] = l_run;
+      rec[1] = xch[row] + xch[kPfRows + row];
     }
   } else {
     // a bounded wait gave up: drain what the tensor cores and the bulk copy
@@ -495,7 +521,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const Prefill
       if (p.status != nullptr) atomicOr(p.status, drained ? LOOPVQ_DECODE_STATUS_TIMEOUT
                                                           : (LOOPVQ_DECODE_STATUS_TIMEOUT | LOOPVQ_DECODE_STATUS_UNDRAINED));
     }
-    if (row_ok) {
+    if (row_ok && colh == 0) {
       rec[0] = NAN;
       rec[1] = 1.f;
     }
@@ -526,7 +552,7 @@ size_t prefill_tc_workspace_bytes(const Geometry& g, int batch, int n_queries, i
   if (CH != nullptr) *CH = ch;
   const size_t rows = static_cast<size_t>(batch) * n_queries * g.Hq;
   const size_t rec = rows * s * (g.d + 2) * sizeof(float);
-  const size_t cb = static_cast<size_t>(g.Hkv) * kCb16Elems * 2;
+  const size_t cb = static_cast<size_t>(g.Hkv) * kCb16Elems * 2 * 3;   // value bf16, key hi/lo
   return kStatusBytes + ((rec + 255) / 256) * 256 + cb;
 }
 
@@ -550,8 +576,7 @@ loopvq_status launch_prefill_tc(const DecodeArgs& a, size_t workspace_bytes) {
   const size_t rec = rows * S * (g.d + 2) * sizeof(float);
   uint16_t* cb16 = reinterpret_cast<uint16_t*>(ws + kStatusBytes + ((rec + 255) / 256) * 256);
   p.cbv16 = cb16;
-  p.cb_k = cb_l;
-  p.cb_stride_head = g.cb_stride_head;
+  p.cbk16 = cb16 + static_cast<size_t>(g.Hkv) * kCb16Elems;
   p.block_table = a.block_table;
   p.seq_lens = a.seq_lens;
   p.win_k = static_cast<const uint16_t*>(a.win_k);
@@ -571,7 +596,8 @@ loopvq_status launch_prefill_tc(const DecodeArgs& a, size_t workspace_bytes) {
   p.QT = (a.n_queries + kPfRows - 1) / kPfRows;
   p.scale_log2 = a.sm_scale * kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(a.stream);
-  prefill_cb_kernel<<<g.Hkv * 2, 256, 0, st>>>(cb_l + g.cb_stride_kv, g.cb_stride_head, g.Hkv, cb16);
+  prefill_cb_kernel<<<g.Hkv * 2, 256, 0, st>>>(cb_l, cb_l + g.cb_stride_kv, g.cb_stride_head, g.Hkv, cb16,
+                                               cb16 + static_cast<size_t>(g.Hkv) * kCb16Elems);
   if (cudaGetLastError() != cudaSuccess) return LOOPVQ_ERR_CUDA;
   static_assert(kPfSmem <= 227 * 1024, "prefill shared memory above 227 KB");
   if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem) != cudaSuccess)
