@@ -347,9 +347,19 @@ loopvq_status loopvq_decode_attn(const loopvq_config* cfg, int layer, int loop_s
  *  lse    float32 [batch][n_queries][Hq] or NULL.
  *  workspace  at least loopvq_prefill_workspace_bytes(cfg, batch, n_queries,
  *         max_seq_len) bytes; the status word as for loopvq_decode_attn.
- * Every other argument as for loopvq_decode_attn. The queries of a
- * sequence are streamed by neighbouring CTAs, so each index page crosses
- * HBM about once and is reused from L2.
+ * Every other argument as for loopvq_decode_attn.
+ *
+ * Two forms, chosen per call:
+ *  - bf16 output, n_queries >= 64, head_dim 128 and chan_group 4: the
+ *    tensor-core form. Each tile of 64 tokens is dequantised once for a tile
+ *    of 128 queries and both products run on the tensor cores; the key
+ *    codewords enter in two bf16 parts (scores and lse keep float32-level
+ *    precision), the value codewords and softmax weights in bf16 (about
+ *    2^-9 relative in the output). A bounded wait that gives up sets
+ *    LOOPVQ_DECODE_STATUS_TIMEOUT (and _UNDRAINED) in the status word.
+ *  - otherwise: the decode kernels over batch*n_queries virtual sequences
+ *    (neighbouring CTAs share each sequence's pages through L2), exact in
+ *    float32 like loopvq_decode_attn.
  */
 size_t loopvq_prefill_workspace_bytes(const loopvq_config* cfg, int batch, int n_queries,
                                       int max_seq_len);
