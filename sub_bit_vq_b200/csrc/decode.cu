@@ -23,8 +23,11 @@
 //      one byte permute plus the immediate 4s; the scores x (log2 units) stay
 //      in registers. The warps' maxima and weight sums meet at a barrier,
 //      which fixes the segment's integer reference maximum m (raised to
-//      ceil(max x)) and its fixed-point exponent S. Value phase, lane = slot
-//      again: the slot's weight w = rn(2^(x - m + S)) is added to cell
+//      ceil(max x) + 1 when a chunk passes it) and its fixed-point exponent
+//      S. Value phase, lane = slot again: the slot's weight
+//      w = rn(2^(x - cm) * 2^(cm - m + S)) = rn(2^(x - m + S)) (cm: the
+//      warp's chunk maximum, whose powers 2^(x - cm) also gave the weight
+//      sums) is added to cell
 //      H[idx][lane + s] for each byte s of its rotated V row by a 32-bit
 //      shared-memory reduction (red.shared.add.u32: integer reductions run
 //      at full shared-memory rate on sm_100, so all warps update the one
@@ -32,15 +35,17 @@
 //      Overflow: every cell is a sum of weights of distinct tokens, so it
 //      never exceeds the total weight of the segment, which the barrier
 //      knows exactly. S starts at kFixMax and is lowered whenever that total
-//      would pass 2^31; m rises when a chunk's maximum passes it. Either
-//      change is an exact right shift of every cell by the bits lost.
+//      would pass 2^31 (the total then lands below 2^29); m rises only when
+//      a chunk's maximum passes it. Either change is an exact right shift of
+//      every cell by the bits lost.
 //   3. The histogram, converted to float (W[e][j] = 2^-S sum of the columns
 //      of group j), is contracted with the value codebook slice,
 //      o_j = sum_e W[e][j] C_V[j][e][tau], and the segment record
 //      (m, l = sum_e W[e][j], o[d]) goes to slot (pair + cta).
 //   4. The CTA counts its record on the pair's counter; the CTA that writes
 //      the pair's last record merges the window partial with every record
-//      (log-sum-exp weights) and writes out and lse. No CTA waits on another.
+//      (log-sum-exp weights, one round of loads per channel) and writes out
+//      and lse. No CTA waits on another.
 //
 // The hot loops address shared memory by absolute shared-window address: a
 // byte permute puts an index byte into byte 1 of (lane * 4), and the window
@@ -72,6 +77,10 @@ constexpr int kPairThreads = 256;         // window partial: 8 warps; lookup tab
 constexpr int kWinChunk = 9;              // window tokens per warp per round of loads (72 = 8 warps x 9)
 constexpr int kSegmentUnits = 16;         // work units (pages) charged for a segment's setup
 constexpr int kCols = 64;                 // columns of the shared LUT and histogram
+constexpr float kMHead = 1.f;             // headroom of the reference maximum, log2 units
+constexpr int kPsBits = 24;               // fixed-point bits of a warp's chunk weight sum
+constexpr int kAddBits = 20;              // fixed-point bits of the CTA's chunk weight sum
+constexpr float kPsScale = 16777216.0f;   // 2^kPsBits
 
 // Shared memory, by absolute shared-window address. The dynamic allocation
 // starts at kSBase (the reserved shared memory of a block on sm_100).
@@ -222,6 +231,36 @@ template <uint32_t OFF>
 __device__ __forceinline__ void red_at(uint32_t a, uint32_t w) {
   asm volatile("red.shared.add.u32 [%0+%1], %2;" ::"r"(a), "n"(OFF), "r"(w));
 }
+
+// Warp-wide maximum (NaN ignored) and unsigned sum, one instruction each.
+__device__ __forceinline__ float redux_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t redux_add_u32(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.add.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+// Two floats packed in 64 bits (low first), and their lane-wise sum.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// x * 2^k for -126 <= k <= 127, by an exact power-of-two factor.
+__device__ __forceinline__ float ldexp_pos(float x, int k) { return x * __int_as_float((127 + k) << 23); }
 
 // Quantised-token pages of sequence b.
 __device__ __forceinline__ int seq_pages(const DecodeParams& p, int b) {
@@ -393,68 +432,60 @@ __device__ void window_partial(const DecodeParams& p, int b, int hkv, const uint
 // Merges a pair's window partial with its segment records (slots pair + c
 // for the CTAs c in [c_first, c_last] whose unit range is not empty: CTA c
 // of n_cta owns units [U*c/n_cta, U*(c+1)/n_cta)) and writes out and lse.
-// Every thread of the CTA (NT threads) calls it; sh holds 4 + 256 floats.
-// m in log2 units; a record with m = -inf is empty, a NaN m poisons the
-// result.
+// Every thread of the CTA (NT threads) calls it. Thread ch owns output
+// channel ch: it loads (m, l, o[ch]) of the window partial and of up to
+// kMergeBatch records at once and folds them in with log-sum-exp weights,
+// so that one round of loads serves every pair that spans at most
+// kMergeBatch CTAs (all but the smallest batches). m in log2 units; a record
+// with m = -inf is empty, a NaN m poisons the result.
 template <int D, int NT>
-__device__ void merge_pair(const DecodeParams& p, int pair, int c_first, int c_last, long long U,
-                           float* sh) {
+__device__ void merge_pair(const DecodeParams& p, int pair, int c_first, int c_last, long long U) {
   constexpr int RS = 4 + D;
-  const int tid = threadIdx.x, lane = tid & 31;
+  constexpr int kMergeBatch = 8;
   const float* wr = p.wrecs + static_cast<size_t>(pair) * RS;
   const bool every = U >= p.n_cta;                     // then no CTA's range is empty
   auto written = [&](int c) { return every || U * c / p.n_cta < U * (c + 1) / p.n_cta; };
-  if (tid < 32) {
-    // (m, l) of the window partial and of up to 32 records per round, loaded together
-    const float m_win = __ldcg(wr), l_win = __ldcg(wr + 1);
-    float M = m_win;
-    float mc[8], lc[8];
+  for (int ch = threadIdx.x; ch < D; ch += NT) {
+    const float m_win = __ldcg(wr), l_win = __ldcg(wr + 1), o_win = __ldcg(wr + 4 + ch);
+    float m = m_win, l = 0.f, o = 0.f;
+    if (m_win != -INFINITY) {
+      l = l_win;
+      o = o_win;
+    }
+    for (int c0 = c_first; c0 <= c_last; c0 += kMergeBatch) {
+      float mc[kMergeBatch], lc[kMergeBatch], oc[kMergeBatch];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int c = c_first + lane + 32 * r;
-      mc[r] = -INFINITY;
-      lc[r] = 0.f;
-      if (c <= c_last && written(c)) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.records + static_cast<size_t>(pair + c) * RS));
-        mc[r] = ml.x;
-        lc[r] = ml.y;
+      for (int r = 0; r < kMergeBatch; ++r) {
+        const int c = c0 + r;
+        mc[r] = -INFINITY;
+        lc[r] = oc[r] = 0.f;
+        if (c <= c_last && written(c)) {
+          const float* rc = p.records + static_cast<size_t>(pair + c) * RS;
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(rc));
+          mc[r] = ml.x;
+          lc[r] = ml.y;
+          oc[r] = __ldcg(rc + 4 + ch);
+        }
       }
-      M = fmaxf(M, mc[r]);
-    }
-    M = warp_max(M);
-    float L = 0.f;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int c = c_first + lane + 32 * r;
-      const float f = (mc[r] == -INFINITY) ? 0.f : fast_exp2(mc[r] - M);   // a NaN m poisons M and L
-      L += lc[r] * f;
-      if (c <= c_last) sh[4 + c - c_first] = f;
+      for (int r = 0; r < kMergeBatch; ++r) {
+        if (mc[r] == -INFINITY) continue;              // empty record
+        const float mn = fmaxf(m, mc[r]);              // a NaN mc gives NaN factors below
+        const float f0 = (m == -INFINITY) ? 0.f : fast_exp2(m - mn);
+        const float f1 = fast_exp2(mc[r] - mn);
+        l = fmaf(l, f0, lc[r] * f1);
+        o = fmaf(o, f0, oc[r] * f1);
+        m = mn;
+      }
     }
-    L = warp_sum(L);
-    if (lane == 0) {
-      const float f_win = (m_win == -INFINITY) ? 0.f : fast_exp2(m_win - M);
-      sh[0] = M;
-      sh[1] = L + f_win * l_win;
-      sh[2] = f_win;
-    }
-  }
-  __syncthreads();
-  const float M = sh[0], L = sh[1], f_win = sh[2];
-  const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  for (int ch = tid; ch < D; ch += NT) {
-    float o = (f_win != 0.f) ? f_win * __ldcg(wr + 4 + ch) : 0.f;
-    for (int c = c_first; c <= c_last; ++c) {
-      const float f = sh[4 + c - c_first];
-      if (f != 0.f) o = fmaf(f, __ldcg(p.records + static_cast<size_t>(pair + c) * RS + 4 + ch), o);
-    }
-    o *= inv;
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const float v = o * inv;
     if (p.out_dtype == LOOPVQ_DTYPE_F32)
-      static_cast<float*>(p.out)[static_cast<size_t>(pair) * D + ch] = o;
+      static_cast<float*>(p.out)[static_cast<size_t>(pair) * D + ch] = v;
     else
-      static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(pair) * D + ch] = __float2bfloat16_rn(o);
+      static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(pair) * D + ch] = __float2bfloat16_rn(v);
+    if (ch == 0 && p.lse != nullptr) p.lse[pair] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
   }
-  if (tid == 0 && p.lse != nullptr)
-    p.lse[pair] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
 }
 
 // The per-pair work that needs no index stream, before the streaming
@@ -487,7 +518,7 @@ __global__ void __launch_bounds__(kPairThreads) vq_pair_kernel(const DecodeParam
     if (tid == 0) p.counts[pair] = 0u;
     if (seq_pages(p, b) == 0) {                        // window tokens only: the result is final here
       __syncthreads();
-      merge_pair<D, kPairThreads>(p, pair, 0, -1, 1, wpart);
+      merge_pair<D, kPairThreads>(p, pair, 0, -1, 1);
     }
     return;
   }
@@ -612,7 +643,17 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       const int n_blocks = n_my_pages << lbpp;
       const int n_chunks = ((pages_of(0) << lbpp) + KB - 1) / KB;   // CTA-uniform (warp 0 has the most)
       int i0 = 0;                                      // page-table window: this warp's pages [i0, i0 + 64)
-      auto bt_entry = [&](int i) -> int { return (i < n_my_pages) ? bt[my_first + i * kNW] : -1; };
+      // page-table entry of this warp's page i, or -1 past its pages; an entry
+      // outside the pool flags the status word and reads as -1 (its blocks are
+      // skipped)
+      auto bt_entry = [&](int i) -> int {
+        int v = (i < n_my_pages) ? bt[my_first + i * kNW] : -1;
+        if (i < n_my_pages && (v < 0 || v >= p.n_pages)) {
+          if (p.status != nullptr) atomicOr(p.status, kStatusBadPage);
+          v = -1;
+        }
+        return v;
+      };
       int bt_cur = bt_entry(lane);
       int bt_nxt = bt_entry(32 + lane);
       // L2 prefetch of pages [k0, k1) of this warp's list
@@ -629,23 +670,20 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       BlockRegs<J> ring[kRing];
       BlockInfo info[KB];
       // Locates block t of this warp (its key row is loaded by the caller).
+      // No branch: a block past this warp's list or on a skipped page gets
+      // nv = 0 and the row of page 0 (in the pool, never read for nv = 0).
       auto locate = [&](int t, BlockInfo& bi) {
-        bi.nv = 0;
-        if (t >= n_blocks) return;                     // warp-uniform
         const int pi = t >> lbpp, blk = t & (bpp - 1);
         const int src = (pi - i0 < 32) ? bt_cur : bt_nxt;
         const int phys = __shfl_sync(0xffffffffu, src, (pi - i0) & 31);
-        if (phys < 0 || phys >= p.n_pages) {           // a page-table entry outside the pool
-          if (lane == 0 && p.status != nullptr) atomicOr(p.status, kStatusBadPage);
-          return;
-        }
         const int pg = my_first + pi * kNW;
-        if (kRangeCheck && (pg < 0 || pg >= p.max_pages_per_seq || blk >= bpp)) {
+        bool ok = t < n_blocks && phys >= 0;
+        if (kRangeCheck && ok && (pg < 0 || pg >= p.max_pages_per_seq || blk >= bpp)) {
           if (lane == 0 && p.status != nullptr) atomicOr(p.status, LOOPVQ_DECODE_STATUS_RANGE);
-          return;
+          ok = false;
         }
-        bi.nv = max(0, min(LB, n_vq - pg * p.Pg - blk * LB));
-        bi.row = pool_h + static_cast<int64_t>(phys) * p.page_bytes + blk * (LB * J) + lane * T::GR;
+        bi.nv = ok ? max(0, min(LB, n_vq - pg * p.Pg - blk * LB)) : 0;
+        bi.row = pool_h + (ok ? static_cast<int64_t>(phys) * p.page_bytes + blk * (LB * J) : 0) + lane * T::GR;
       };
       // the key rows of chunk ch into the ring (and their locations into info)
       auto issue_keys = [&](int ch) {
@@ -694,21 +732,26 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       }
       __syncthreads();                                 // LUT and histogram ready, staging area free
       // ---- stream -------------------------------------------------------------
+      // every block is scored (a block with nv = 0 holds stale or zero bytes,
+      // which address cells inside the table) and masked afterwards
       auto key_score = [&](const BlockRegs<J>& r, int nv) -> float {
-        if (nv <= 0) return -INFINITY;                 // warp-uniform
         uint32_t ad[J];
 #pragma unroll
         for (int s = 0; s < J; ++s) ad[s] = __byte_perm(r.w[s >> 2], lane4, 0x7604u | (uint32_t(s & 3) << 4));
-        float xa[4] = {0.f, 0.f, 0.f, 0.f};
-        constexpr_for<J>([&](auto S) { xa[S.value & 3] += lds_at<kLutAbs + 4u * S.value>(ad[S.value]); });
-        return lane < nv ? (xa[0] + xa[1]) + (xa[2] + xa[3]) : -INFINITY;
+        uint64_t xa[2] = {0ull, 0ull};                 // two packed pairs of partial sums
+        constexpr_for<J / 2>([&](auto P) {
+          constexpr int s = 2 * P.value;
+          xa[P.value & 1] = add_f32x2(xa[P.value & 1], f2_pack(lds_at<kLutAbs + 4u * s>(ad[s]),
+                                                                  lds_at<kLutAbs + 4u * (s + 1)>(ad[s + 1])));
+        });
+        const float2 a = f2_unpack(xa[0]), b = f2_unpack(xa[1]);
+        return lane < nv ? (a.x + a.y) + (b.x + b.y) : -INFINITY;
       };
       // histogram updates of one value block, lane = slot: the slot's weight
       // w = rn(2^(x - m + S)) goes to cell [idx][lane + s] for each byte s of its
       // rotated value row (w = 0 for an invalid slot)
-      auto value_pass = [&](const BlockRegs<J>& r, int nv, float x, float mS) {
-        if (nv <= 0) return;                           // warp-uniform
-        const uint32_t w = __float2uint_rn(fast_exp2(x - mS));
+      auto value_pass = [&](const BlockRegs<J>& r, float ex, float factor) {
+        const uint32_t w = __float2uint_rn(ex * factor);
         uint32_t ad[J];
 #pragma unroll
         for (int s = 0; s < J; ++s) ad[s] = __byte_perm(r.w[s >> 2], lane4, 0x7604u | (uint32_t(s & 3) << 4));
@@ -740,13 +783,17 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           cm = fmaxf(cm, xs[q]);
           issue_value(q);
         }
-        cm = warp_max(cm);
-        float ps = 0.f;                                // sum of 2^(x - cm) over this warp's slots
-        if (cm != -INFINITY) {                         // warp-uniform
+        cm = redux_max(cm);
+        // xs[q] becomes 2^(x - cm) (0 for an invalid slot, and for every slot
+        // of a warp without a valid one); ps sums them over the warp in units
+        // of 2^-kPsBits (a lane's share is at most KB, so the sum fits 32 bits)
+        float ps = 0.f;
 #pragma unroll
-          for (int q = 0; q < KB; ++q) ps += fast_exp2(xs[q] - cm);   // 0 for x = -inf
-          ps = warp_sum(ps);
+        for (int q = 0; q < KB; ++q) {
+          xs[q] = (cm == -INFINITY) ? 0.f : fast_exp2(xs[q] - cm);
+          ps += xs[q];
         }
+        ps = ldexp_pos(redux_add_u32(__float2uint_rn(ps * kPsScale)), -kPsBits);
         float* st = stat + (ch & 1) * 2 * kNW;
         if (lane == 0) {
           st[2 * warp] = cm;
@@ -754,15 +801,19 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         }
         __syncthreads();                               // every warp's chunk maximum and sum
         const float cmw = (lane < kNW) ? st[2 * lane] : -INFINITY;
-        const float cmax = warp_max(cmw);
+        const float cmax = redux_max(cmw);
         if (cmax != -INFINITY) {                       // CTA-uniform
-          const float m_new = fmaxf(m_cur, ceilf(cmax));
+          // m rises to ceil(max) + kMHead, so that a later chunk passes it (and
+          // costs a rescale) only when its maximum is a whole unit higher
+          const float m_new = (cmax > m_cur) ? ceilf(cmax) + kMHead : m_cur;
+          // the chunk's weights in units of 2^m_new, summed in fixed point (a
+          // warp's share is at most 32 * KB)
           const float psw = (lane < kNW && cmw != -INFINITY) ? st[2 * lane + 1] * fast_exp2(cmw - m_new) : 0.f;
-          const float add = warp_sum(psw);             // the chunk's weights, units of 2^m_new
+          const float add = ldexp_pos(redux_add_u32(__float2uint_rn(ldexp_pos(psw, kAddBits))), -kAddBits);
           const float kept = (m_cur == -INFINITY) ? 0.f : mass * fast_exp2(m_cur - m_new);
           const float total = kept + add;
           int S_new = S;
-          if (ldexpf(total, S) + static_cast<float>(kThreads * KB) > kMassHigh) {
+          if (ldexp_pos(total, S) + static_cast<float>(kThreads * KB) > kMassHigh) {
             int ex;
             frexpf(total, &ex);                        // total < 2^ex
             S_new = min(S, kMassLandLog2 - ex);
@@ -776,10 +827,11 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
           S = S_new;
           mass = total;
         }
-        const float mS = m_cur - static_cast<float>(S);
+        // w = rn(2^(x - m + S)) = rn(2^(x - cm) * 2^(cm - m + S)); 0 for an invalid slot
+        const float factor = (cm == -INFINITY || m_cur == -INFINITY) ? 0.f : fast_exp2(cm - m_cur + static_cast<float>(S));
 #pragma unroll
         for (int q = 0; q < KB; ++q) {                 // value phase
-          if (m_cur != -INFINITY) value_pass(ring[q], info[q].nv, xs[q], mS);   // CTA-uniform
+          value_pass(ring[q], xs[q], factor);
           if (q == 0) issue_keys(ch + 1);
           issue_key(ch + 1, q);
         }
@@ -877,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       __syncthreads();
       if (*s_last) {                                   // CTA-uniform: every record of the pair is written
         __threadfence();
-        merge_pair<d, kThreads>(p, pair, c_first, c_last, U, lut);
+        merge_pair<d, kThreads>(p, pair, c_first, c_last, U);
       }
     }
 
