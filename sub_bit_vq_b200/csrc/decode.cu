@@ -775,13 +775,27 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
       float mass = 0.f;                                // sum of weights so far, units of 2^(m_cur) (CTA-uniform)
 #pragma unroll 1
       for (int ch = 0; ch < n_chunks; ++ch) {
+        // A chunk whose last block is past this warp's pages (the last chunk
+        // of a warp with fewer pages than warp 0) skips its empty blocks;
+        // every other chunk runs without a branch per block (an empty block
+        // there, on a skipped page, is reduced with weight 0).
+        const bool tail = !__all_sync(0xffffffffu, info[KB - 1].nv > 0);   // warp-uniform
         float xs[KB];
         float cm = -INFINITY;
+        if (!tail) {
 #pragma unroll
-        for (int q = 0; q < KB; ++q) {                 // key phase
-          xs[q] = key_score(ring[q], info[q].nv);
-          cm = fmaxf(cm, xs[q]);
-          issue_value(q);
+          for (int q = 0; q < KB; ++q) {               // key phase
+            xs[q] = key_score(ring[q], info[q].nv);
+            cm = fmaxf(cm, xs[q]);
+            issue_value(q);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < KB; ++q) {
+            xs[q] = (info[q].nv > 0) ? key_score(ring[q], info[q].nv) : -INFINITY;
+            cm = fmaxf(cm, xs[q]);
+            issue_value(q);
+          }
         }
         cm = redux_max(cm);
         // xs[q] becomes 2^(x - cm) (0 for an invalid slot, and for every slot
@@ -829,11 +843,20 @@ __global__ void __launch_bounds__(kThreads, 1) vq_stream_kernel(const DecodePara
         }
         // w = rn(2^(x - m + S)) = rn(2^(x - cm) * 2^(cm - m + S)); 0 for an invalid slot
         const float factor = (cm == -INFINITY || m_cur == -INFINITY) ? 0.f : fast_exp2(cm - m_cur + static_cast<float>(S));
+        if (!tail) {
 #pragma unroll
-        for (int q = 0; q < KB; ++q) {                 // value phase
-          value_pass(ring[q], xs[q], factor);
-          if (q == 0) issue_keys(ch + 1);
-          issue_key(ch + 1, q);
+          for (int q = 0; q < KB; ++q) {               // value phase
+            value_pass(ring[q], xs[q], factor);
+            if (q == 0) issue_keys(ch + 1);
+            issue_key(ch + 1, q);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < KB; ++q) {
+            if (info[q].nv > 0) value_pass(ring[q], xs[q], factor);
+            if (q == 0) issue_keys(ch + 1);
+            issue_key(ch + 1, q);
+          }
         }
       }
       __syncthreads();                                 // every update landed
