@@ -69,7 +69,7 @@ constexpr int kNW = 16;                   // warps of the streaming kernel
 constexpr int kThreads = kNW * 32;
 constexpr int kRing = 4;                  // index blocks in registers
 constexpr int kChunkBlocks = 4;           // blocks per warp per chunk (key phase, then value phase)
-constexpr int kPrefetchPages = 4;         // pages a warp asks L2 to fetch ahead of its loads
+constexpr int kPrefetchPages = 2;         // pages a warp asks L2 to fetch ahead of its loads
 constexpr int kFixMax = 30;               // largest fixed-point exponent: w = rn(2^(x - m) * 2^S)
 constexpr float kMassHigh = 2147483648.0f;  // 2^31: lower S before a segment's total passes this
 constexpr int kMassLandLog2 = 29;         // after lowering S the total sits below 2^29
